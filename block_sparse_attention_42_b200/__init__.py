@@ -1,0 +1,10 @@
+"""B200-native (sm_100a) Stem block-sparse prefill: OAM scoring, TPD selection, block-sparse
+causal attention.  The kernels and the C ABI live in libbsa.so (``build.build()`` compiles
+it in-tree); this package exposes the ABI's entry points through ``binding``."""
+from .binding import (BSA_BF16, BSA_FP8_E4M3, BSA_FP32, BSA_METRIC_OAM, BSA_METRIC_OAM_MUL, BSA_METRIC_SAM,
+                      BsaError, bsa_check_device_error, bsa_prefill, bsa_prefill_paged, bsa_score_workspace_bytes,
+                      bsa_tpd_budget, stem_score, stem_select)
+
+__all__ = ["stem_score", "stem_select", "bsa_prefill", "bsa_prefill_paged", "bsa_tpd_budget",
+           "bsa_score_workspace_bytes", "bsa_check_device_error", "BsaError", "BSA_BF16", "BSA_FP8_E4M3",
+           "BSA_FP32", "BSA_METRIC_OAM", "BSA_METRIC_SAM", "BSA_METRIC_OAM_MUL"]

@@ -1,0 +1,197 @@
+"""Thin ctypes binding of libbsa.so: the same entry points as include/bsa.h.
+
+Argument marshalling only: torch tensors become pointers, strides and the current CUDA
+stream; every step of the path runs in the library's kernels.  PyTorch allocates outputs
+and workspaces when the caller passes none.  There is no fallback: if libbsa.so is missing
+or fails to load, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+from pathlib import Path
+
+import torch
+
+_LIB_PATH = Path(__file__).resolve().parent / "libbsa.so"
+_lib = None
+
+BSA_BF16, BSA_FP8_E4M3, BSA_FP32 = 0, 1, 2
+BSA_METRIC_OAM, BSA_METRIC_SAM, BSA_METRIC_OAM_MUL = 0, 1, 2
+STATUS = {0: "BSA_OK", 1: "BSA_ERR_INVALID_ARG", 2: "BSA_ERR_UNSUPPORTED", 3: "BSA_ERR_CUDA",
+          4: "BSA_ERR_WORKSPACE", 5: "BSA_ERR_INVALID_LIST", 6: "BSA_ERR_TIMEOUT"}
+
+# Every symbol include/bsa.h declares.
+EXPORTS = ["bsa_tpd_budget", "bsa_score_workspace_bytes", "stem_score", "stem_select", "bsa_prefill",
+           "bsa_prefill_paged", "bsa_last_error", "bsa_check_device_error"]
+
+
+class BsaError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+class BsaTensor(ctypes.Structure):
+    _fields_ = [("ptr", ctypes.c_void_p), ("dtype", ctypes.c_int32), ("scale", ctypes.c_float),
+                ("stride_b", ctypes.c_int64), ("stride_t", ctypes.c_int64), ("stride_h", ctypes.c_int64)]
+
+
+def lib():
+    """Loads libbsa.so (raises if it is missing: there is no CPU or library fallback)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not _LIB_PATH.exists():
+        raise ImportError(f"{_LIB_PATH.name} is not built; run block_sparse_attention_42_b200.build.build()")
+    L = ctypes.CDLL(str(_LIB_PATH))
+    P, i32, i64, f32, f64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_double
+    T = BsaTensor
+    L.bsa_tpd_budget.argtypes = [i32, f64, f64, P]
+    L.bsa_tpd_budget.restype = i64
+    L.bsa_score_workspace_bytes.argtypes = [i32, i32, i32, i32, i32]
+    L.bsa_score_workspace_bytes.restype = ctypes.c_size_t
+    L.stem_score.argtypes = [T, T, T, i32, i32, i32, i32, i32, i32, i32, f32, P, i32, P, ctypes.c_size_t, P]
+    L.stem_select.argtypes = [P, i32, i32, P, i32, f64, f64, P, P, i64, P]
+    L.bsa_prefill.argtypes = [T, T, T, T, i32, i32, i32, i32, i32, i32, P, i32, P, i64, f32, P, P]
+    L.bsa_prefill_paged.argtypes = [T, T, P, P, i32, T, T, i32, i32, P, i32, i32, i32, i32, i32, P, i32, P, i64,
+                                    f32, P, P]
+    L.bsa_last_error.restype = ctypes.c_char_p
+    L.bsa_check_device_error.argtypes = [P]
+    for name in ["stem_score", "stem_select", "bsa_prefill", "bsa_prefill_paged", "bsa_check_device_error"]:
+        getattr(L, name).restype = ctypes.c_int
+    _lib = L
+    return L
+
+
+def _check(status: int):
+    if status != 0:
+        raise BsaError(status, lib().bsa_last_error().decode())
+
+
+def _stream(t: torch.Tensor):
+    return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    try:
+        return {torch.bfloat16: BSA_BF16, torch.float8_e4m3fn: BSA_FP8_E4M3, torch.float32: BSA_FP32}[t.dtype]
+    except KeyError:
+        raise TypeError(f"unsupported dtype {t.dtype}") from None
+
+
+def tensor_arg(t: torch.Tensor, scale: float = 1.0) -> BsaTensor:
+    """[B, N, H, d] (or packed [T, H, d]) tensor -> bsa_tensor_t.  The last dim must be contiguous."""
+    if t.stride(-1) != 1:
+        raise ValueError("the head_dim dimension must be contiguous")
+    if t.dim() == 4:
+        sb, st, sh = t.stride()[:3]
+    elif t.dim() == 3:
+        sb, (st, sh) = 0, t.stride()[:2]
+    else:
+        raise ValueError("expected a 4-D [B, N, H, d] or 3-D [T, H, d] tensor")
+    return BsaTensor(t.data_ptr(), _dtype_code(t), float(scale), sb, st, sh)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def bsa_tpd_budget(nb: int, density: float, tpd_decay: float = 0.5):
+    """Host TPD budget: (k [nb] int32 tensor, total)."""
+    k = torch.zeros(max(nb, 1), dtype=torch.int32)
+    tot = lib().bsa_tpd_budget(nb, float(density), float(tpd_decay), ctypes.c_void_p(k.data_ptr()))
+    if tot < 0:
+        raise BsaError(1, "invalid TPD arguments")
+    return k[:nb], int(tot)
+
+
+def bsa_score_workspace_bytes(B, Hq, Hkv, nb, d) -> int:
+    return int(lib().bsa_score_workspace_bytes(B, Hq, Hkv, nb, d))
+
+
+def stem_score(q, k, v, block: int, metric: int = BSA_METRIC_OAM, softmax_scale: float = 0.0, scores=None,
+               nb_stride: int | None = None, workspace=None, q_scale=1.0, k_scale=1.0, v_scale=1.0):
+    """OAM block scores [B, Hq, nb_stride, nb_stride] fp32 (causal lower triangle valid)."""
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    nb = (N + block - 1) // block
+    nbs = nb if nb_stride is None else nb_stride
+    if scores is None:
+        scores = torch.empty(B, Hq, nbs, nbs, dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(bsa_score_workspace_bytes(B, Hq, Hkv, nb, d), dtype=torch.uint8, device=q.device)
+    st = lib().stem_score(tensor_arg(q, q_scale), tensor_arg(k, k_scale), tensor_arg(v, v_scale), B, N, Hq, Hkv, d,
+                          block, metric, float(softmax_scale), _ptr(scores), nbs, _ptr(workspace),
+                          workspace.numel(), _stream(q))
+    _check(st)
+    return scores
+
+
+def stem_select(scores, nb_per_seq, density: float, tpd_decay: float = 0.5, row_ptr=None, col_idx=None,
+                max_k: int | None = None):
+    """TPD budget + top-k: (row_ptr [B, nbs+1], col_idx [B, Hq, max_k]) int32 device tensors."""
+    B, Hq, nbs, _ = scores.shape
+    nbp = torch.tensor(list(nb_per_seq), dtype=torch.int32)
+    if max_k is None:
+        max_k = max(bsa_tpd_budget(int(n), density, tpd_decay)[1] for n in nbp)
+    if row_ptr is None:
+        row_ptr = torch.empty(B, nbs + 1, dtype=torch.int32, device=scores.device)
+    if col_idx is None:
+        col_idx = torch.empty(B, Hq, max_k, dtype=torch.int32, device=scores.device)
+    st = lib().stem_select(_ptr(scores), B, Hq, ctypes.c_void_p(nbp.data_ptr()), nbs, float(density),
+                           float(tpd_decay), _ptr(row_ptr), _ptr(col_idx), int(max_k), _stream(scores))
+    _check(st)
+    return row_ptr, col_idx
+
+
+def bsa_prefill(q, k, v, block: int, row_ptr, col_idx, softmax_scale: float = 0.0, out=None, lse=None,
+                return_lse: bool = False, q_scale=1.0, k_scale=1.0, v_scale=1.0):
+    """Block-sparse causal prefill.  q [B,N,Hq,d], k/v [B,N,Hkv,d]; returns out (BF16)[, lse]."""
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    if out is None:
+        out = torch.empty(B, N, Hq, d, dtype=torch.bfloat16, device=q.device)
+    if return_lse and lse is None:
+        lse = torch.empty(B, Hq, N, dtype=torch.float32, device=q.device)
+    st = lib().bsa_prefill(tensor_arg(q, q_scale), tensor_arg(k, k_scale), tensor_arg(v, v_scale), tensor_arg(out),
+                           B, N, Hq, Hkv, d, block, _ptr(row_ptr), row_ptr.shape[-1], _ptr(col_idx),
+                           col_idx.shape[-1], float(softmax_scale), _ptr(lse), _stream(q))
+    _check(st)
+    return (out, lse) if return_lse else out
+
+
+def bsa_prefill_paged(q, cu_seqlens, seqlens, k_cache, v_cache, page_table, block: int, row_ptr, col_idx,
+                      softmax_scale: float = 0.0, out=None, lse=None, return_lse: bool = False, q_scale=1.0,
+                      k_scale=1.0, v_scale=1.0):
+    """Paged-KV variant: q packed [sum N, Hq, d]; k_cache/v_cache [num_pages, page_size, Hkv, d]."""
+    T, Hq, d = q.shape
+    num_pages, page_size, Hkv, _ = k_cache.shape
+    seqlens = [int(s) for s in seqlens]
+    B = len(seqlens)
+    sl = torch.tensor(seqlens, dtype=torch.int32)
+    if out is None:
+        out = torch.empty(T, Hq, d, dtype=torch.bfloat16, device=q.device)
+    if return_lse and lse is None:
+        lse = torch.empty(B, Hq, max(seqlens), dtype=torch.float32, device=q.device)
+    kc, vc = tensor_arg(k_cache, k_scale), tensor_arg(v_cache, v_scale)
+    st = lib().bsa_prefill_paged(tensor_arg(q, q_scale), tensor_arg(out), _ptr(cu_seqlens),
+                                 ctypes.c_void_p(sl.data_ptr()), B, kc, vc, num_pages, page_size, _ptr(page_table),
+                                 page_table.shape[-1], Hq, Hkv, d, block, _ptr(row_ptr), row_ptr.shape[-1],
+                                 _ptr(col_idx), col_idx.shape[-1], float(softmax_scale), _ptr(lse), _stream(q))
+    _check(st)
+    return (out, lse) if return_lse else out
+
+
+def bsa_check_device_error(device=None):
+    """Synchronises the current stream and raises if a kernel recorded an error."""
+    s = torch.cuda.current_stream(device)
+    _check(lib().bsa_check_device_error(ctypes.c_void_p(s.cuda_stream)))
+
+
+def nb_of(N: int, block: int) -> int:
+    return (N + block - 1) // block
+
+
+def default_scale(d: int) -> float:
+    return 1.0 / math.sqrt(d)

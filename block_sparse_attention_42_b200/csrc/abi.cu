@@ -1,0 +1,431 @@
+// abi.cu -- the extern "C" entry points of libbsa.so declared in include/bsa.h: argument
+// validation (synchronous, nothing launched on error), workspace carving, TMA descriptor
+// encoding and kernel launches.  No device memory is allocated here.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "../../include/bsa.h"
+#include "internal.h"
+
+namespace bsa {
+
+__device__ unsigned g_device_error;  // per-device error word (kDevErr* bits)
+
+namespace {
+
+thread_local std::string g_last_error;
+
+bsa_status_t fail(bsa_status_t st, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return st;
+}
+
+bsa_status_t cuda_fail(cudaError_t e, const char* what) {
+    return fail(BSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+int elt_bytes(int32_t dtype) { return dtype == BSA_BF16 ? 2 : (dtype == BSA_FP8_E4M3 ? 1 : (dtype == BSA_FP32 ? 4 : 0)); }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bsa_status_t check_tensor(const bsa_tensor_t& t, const char* name, bool need_b) {
+    if (t.ptr == nullptr) return fail(BSA_ERR_INVALID_ARG, "%s: null pointer", name);
+    const int eb = elt_bytes(t.dtype);
+    if (eb == 0) return fail(BSA_ERR_INVALID_ARG, "%s: unknown dtype %d", name, t.dtype);
+    if (!aligned16(t.ptr)) return fail(BSA_ERR_INVALID_ARG, "%s: base pointer not 16-byte aligned", name);
+    if (t.stride_t <= 0 || t.stride_h <= 0 || (need_b && t.stride_b <= 0))
+        return fail(BSA_ERR_INVALID_ARG, "%s: strides must be positive", name);
+    if ((t.stride_t * eb) % 16 || (t.stride_h * eb) % 16 || (need_b && (t.stride_b * eb) % 16))
+        return fail(BSA_ERR_INVALID_ARG, "%s: strides must be multiples of 16 bytes", name);
+    if (t.dtype == BSA_FP8_E4M3 && !(t.scale > 0.f && std::isfinite(t.scale)))
+        return fail(BSA_ERR_INVALID_ARG, "%s: FP8 scale must be positive and finite", name);
+    return BSA_OK;
+}
+
+TensorArg targ(const bsa_tensor_t& t) {
+    TensorArg a;
+    a.ptr = t.ptr;
+    a.sb = t.stride_b;
+    a.st = t.stride_t;
+    a.sh = t.stride_h;
+    a.scale = t.dtype == BSA_FP8_E4M3 ? t.scale : 1.f;
+    return a;
+}
+
+unsigned* device_error_word(bsa_status_t* st) {
+    static std::mutex mu;
+    static void* addr[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess || dev < 0 || dev >= 64) {
+        *st = cuda_fail(e, "cudaGetDevice");
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lk(mu);
+    if (addr[dev] == nullptr) {
+        e = cudaGetSymbolAddress(&addr[dev], g_device_error);
+        if (e != cudaSuccess) {
+            addr[dev] = nullptr;
+            *st = cuda_fail(e, "cudaGetSymbolAddress(device error word)");
+            return nullptr;
+        }
+    }
+    *st = BSA_OK;
+    return static_cast<unsigned*>(addr[dev]);
+}
+
+// ---------------------------------------------------------------- TPD budget (host copy)
+
+int64_t tpd_kstar(int32_t nb, double density) {
+    const int64_t T = static_cast<int64_t>(nb) * (nb + 1) / 2;
+    const int64_t sum_m = 2 * static_cast<int64_t>(nb) - 1;
+    int64_t k = static_cast<int64_t>(std::floor(density * static_cast<double>(T) + 0.5));
+    if (k < sum_m) k = sum_m;
+    if (k > T) k = T;
+    return k;
+}
+
+bool tpd_args_ok(int32_t nb, double density, double decay) {
+    return nb >= 1 && nb <= kMaxBlocks * 16 && density > 0.0 && density <= 1.0 && (decay == 0.0 || decay == 0.5);
+}
+
+// ---------------------------------------------------------------- TMA descriptors
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn(bsa_status_t* st) {
+    static std::once_flag once;
+    static EncodeTiledFn fn = nullptr;
+    static cudaError_t err = cudaSuccess;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        err = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+        if (err == cudaSuccess && q == cudaDriverEntryPointSuccess) fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    *st = fn ? BSA_OK : cuda_fail(err == cudaSuccess ? cudaErrorNotSupported : err, "cuTensorMapEncodeTiled lookup");
+    return fn;
+}
+
+// 4-D tiled map over [d, rows, heads, outer] with 128-byte swizzle; box = 128 bytes of d x
+// box_rows x 1 x 1.  Out-of-range boxes read zeros.
+bsa_status_t make_map(CUtensorMap* m, const void* base, int eb, uint64_t d, uint64_t rows, uint64_t heads,
+                      uint64_t outer, int64_t s_rows, int64_t s_heads, int64_t s_outer, uint32_t box_rows,
+                      const char* name) {
+    bsa_status_t st;
+    EncodeTiledFn fn = encode_fn(&st);
+    if (!fn) return st;
+    const cuuint64_t dims[4] = {d, rows, heads, outer};
+    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(s_rows) * eb, static_cast<cuuint64_t>(s_heads) * eb,
+                                   static_cast<cuuint64_t>(s_outer) * eb};
+    const cuuint32_t box[4] = {static_cast<cuuint32_t>(128 / eb), box_rows, 1, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(m, eb == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 4,
+                    const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(BSA_ERR_INVALID_ARG, "%s: cuTensorMapEncodeTiled failed (%d)", name, (int)r);
+    return BSA_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+bsa_status_t attn_common_checks(const bsa_tensor_t& q, const bsa_tensor_t& k, const bsa_tensor_t& v,
+                                const bsa_tensor_t& out, int32_t Hq, int32_t Hkv, int32_t d, int32_t block,
+                                const int32_t* row_ptr, const int32_t* col_idx, int64_t max_k) {
+    if (q.dtype != k.dtype || q.dtype != v.dtype)
+        return fail(BSA_ERR_INVALID_ARG, "q, k and v must share a dtype");
+    if (q.dtype != BSA_BF16 && q.dtype != BSA_FP8_E4M3)
+        return fail(BSA_ERR_UNSUPPORTED, "attention supports BF16 or FP8_E4M3 inputs");
+    if (out.dtype != BSA_BF16) return fail(BSA_ERR_UNSUPPORTED, "out must be BF16");
+    if (Hq < 1 || Hkv < 1 || Hq % Hkv) return fail(BSA_ERR_INVALID_ARG, "Hq must be a positive multiple of Hkv");
+    if (d != 64 && d != 128) return fail(BSA_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
+    if (block != 64 && block != 128) return fail(BSA_ERR_UNSUPPORTED, "block must be 64 or 128");
+    if (q.dtype == BSA_FP8_E4M3 && (d != 128 || block != 128))
+        return fail(BSA_ERR_UNSUPPORTED, "FP8 attention needs head_dim 128 and block 128");
+    if (!row_ptr || !col_idx) return fail(BSA_ERR_INVALID_ARG, "row_ptr/col_idx are null");
+    if (max_k < 1) return fail(BSA_ERR_INVALID_ARG, "max_k must be positive");
+    return BSA_OK;
+}
+
+}  // namespace
+}  // namespace bsa
+
+using namespace bsa;
+
+extern "C" {
+
+int64_t bsa_tpd_budget(int32_t nb, double density, double tpd_decay, int32_t* k_out) {
+    if (!k_out || !tpd_args_ok(nb, density, tpd_decay)) return -1;
+    const int64_t kstar = tpd_kstar(nb, density);
+    const bool half = tpd_decay == 0.5;
+    auto share = [&](double c, int i) -> int64_t {
+        const double n = static_cast<double>(i + 1), m = i == 0 ? 1.0 : 2.0;
+        const double w = half ? std::sqrt(n) : n;
+        volatile double t = c * w;  // one rounding, no contraction
+        double tt = t;
+        if (tt < m) tt = m;
+        if (tt > n) tt = n;
+        volatile double sc = tt * 4294967296.0;
+        return static_cast<int64_t>(std::floor(static_cast<double>(sc)));
+    };
+    const int64_t target = kstar * (int64_t(1) << 32);
+    double lo = 0.0, hi = static_cast<double>(nb);
+    for (int it = 0; it < 64; ++it) {
+        volatile double sum = lo + hi;
+        const double mid = sum * 0.5;
+        int64_t tot = 0;
+        for (int i = 0; i < nb; ++i) tot += share(mid, i);
+        if (tot >= target)
+            hi = mid;
+        else
+            lo = mid;
+    }
+    int64_t whole = 0;
+    struct Rem {
+        uint32_t f;
+        int32_t i;
+    };
+    Rem* rem = new Rem[nb];
+    int nrem = 0;
+    for (int i = 0; i < nb; ++i) {
+        const int64_t F = share(hi, i);
+        k_out[i] = static_cast<int32_t>(F >> 32);
+        whole += k_out[i];
+        if (k_out[i] < i + 1) rem[nrem++] = Rem{static_cast<uint32_t>(F & 0xFFFFFFFFll), i};
+    }
+    int64_t R = kstar - whole;
+    // Partial selection of the R largest fractions (earlier row first on ties).
+    for (int64_t r = 0; r < R && r < nrem; ++r) {
+        int best = static_cast<int>(r);
+        for (int q = static_cast<int>(r) + 1; q < nrem; ++q)
+            if (rem[q].f > rem[best].f || (rem[q].f == rem[best].f && rem[q].i < rem[best].i)) best = q;
+        Rem t = rem[r];
+        rem[r] = rem[best];
+        rem[best] = t;
+        k_out[rem[r].i] += 1;
+    }
+    delete[] rem;
+    return kstar;
+}
+
+size_t bsa_score_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int32_t nb, int32_t d) {
+    if (B < 1 || Hq < 1 || Hkv < 1 || nb < 1 || d < 1) return 0;
+    return align256(sizeof(float) * size_t(B) * Hq * nb * d) + align256(sizeof(float) * size_t(B) * Hkv * nb * d) +
+           align256(sizeof(float) * size_t(B) * Hkv * nb);
+}
+
+bsa_status_t stem_score(bsa_tensor_t q, bsa_tensor_t k, bsa_tensor_t v, int32_t B, int32_t N, int32_t Hq,
+                        int32_t Hkv, int32_t d, int32_t block, int32_t metric, float softmax_scale, float* scores,
+                        int32_t nb_stride, void* ws, size_t ws_bytes, cudaStream_t stream) {
+    bsa_status_t st;
+    if ((st = check_tensor(q, "q", B > 1)) || (st = check_tensor(k, "k", B > 1)) || (st = check_tensor(v, "v", B > 1)))
+        return st;
+    if (q.dtype != k.dtype || q.dtype != v.dtype) return fail(BSA_ERR_INVALID_ARG, "q, k and v must share a dtype");
+    if (B < 1 || N < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv)
+        return fail(BSA_ERR_INVALID_ARG, "bad sizes (B=%d N=%d Hq=%d Hkv=%d)", B, N, Hq, Hkv);
+    if (d != 64 && d != 128) return fail(BSA_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
+    if (block != 64 && block != 128) return fail(BSA_ERR_UNSUPPORTED, "block must be 64 or 128");
+    if (metric < BSA_METRIC_OAM || metric > BSA_METRIC_OAM_MUL) return fail(BSA_ERR_INVALID_ARG, "unknown metric");
+    const int nb = (N + block - 1) / block;
+    if (B > 65535 || Hq > 65535) return fail(BSA_ERR_UNSUPPORTED, "B and Hq must be <= 65535");
+    if (!scores) return fail(BSA_ERR_INVALID_ARG, "scores is null");
+    if (nb_stride < nb) return fail(BSA_ERR_INVALID_ARG, "nb_stride (%d) < number of blocks (%d)", nb_stride, nb);
+    const size_t need = bsa_score_workspace_bytes(B, Hq, Hkv, nb, d);
+    if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u))
+        return fail(BSA_ERR_WORKSPACE, "workspace must be >= %zu bytes and 256-byte aligned", need);
+    float* qbar = static_cast<float*>(ws);
+    float* kbar = reinterpret_cast<float*>(static_cast<char*>(ws) + align256(sizeof(float) * size_t(B) * Hq * nb * d));
+    float* vbar = reinterpret_cast<float*>(reinterpret_cast<char*>(kbar) +
+                                           align256(sizeof(float) * size_t(B) * Hkv * nb * d));
+    const float tau = softmax_scale > 0.f ? softmax_scale : 1.f / std::sqrt(static_cast<float>(d));
+    const int dt = q.dtype == BSA_BF16 ? 0 : (q.dtype == BSA_FP8_E4M3 ? 1 : 2);
+    cudaError_t e = launch_pool(dt, targ(q), targ(k), targ(v), B, N, Hq, Hkv, d, block, qbar, kbar, vbar, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "pool launch");
+    e = launch_score(qbar, kbar, vbar, B, Hq, Hkv, nb, d, tau, metric, scores, nb_stride, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "score launch");
+    return BSA_OK;
+}
+
+bsa_status_t stem_select(const float* scores, int32_t B, int32_t Hq, const int32_t* nb_per_seq, int32_t nb_stride,
+                         double density, double tpd_decay, int32_t* row_ptr, int32_t* col_idx, int64_t max_k,
+                         cudaStream_t stream) {
+    if (!scores || !nb_per_seq || !row_ptr || !col_idx) return fail(BSA_ERR_INVALID_ARG, "null pointer argument");
+    if (B < 1 || B > kMaxBatch) return fail(BSA_ERR_UNSUPPORTED, "B must be in [1, %d]", kMaxBatch);
+    if (Hq < 1) return fail(BSA_ERR_INVALID_ARG, "Hq must be positive");
+    if (nb_stride < 1 || nb_stride > kMaxBlocks)
+        return fail(BSA_ERR_UNSUPPORTED, "nb_stride must be in [1, %d]", kMaxBlocks);
+    if (!(density > 0.0 && density <= 1.0)) return fail(BSA_ERR_INVALID_ARG, "density must be in (0, 1]");
+    if (!(tpd_decay == 0.0 || tpd_decay == 0.5)) return fail(BSA_ERR_UNSUPPORTED, "tpd_decay must be 0 or 0.5");
+    SelectSeqs seqs;
+    seqs.B = B;
+    for (int b = 0; b < B; ++b) {
+        const int nb = nb_per_seq[b];
+        if (nb < 1 || nb > nb_stride) return fail(BSA_ERR_INVALID_ARG, "nb_per_seq[%d]=%d out of [1, nb_stride]", b, nb);
+        seqs.nb[b] = nb;
+        seqs.kstar[b] = tpd_kstar(nb, density);
+        if (seqs.kstar[b] > max_k)
+            return fail(BSA_ERR_INVALID_ARG, "max_k=%lld is below the budget %lld of sequence %d", (long long)max_k,
+                        (long long)seqs.kstar[b], b);
+    }
+    cudaError_t e = launch_select(scores, seqs, Hq, nb_stride, tpd_decay == 0.5, row_ptr, col_idx, max_k, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "select launch");
+    return BSA_OK;
+}
+
+bsa_status_t bsa_prefill(bsa_tensor_t q, bsa_tensor_t k, bsa_tensor_t v, bsa_tensor_t out, int32_t B, int32_t N,
+                         int32_t Hq, int32_t Hkv, int32_t d, int32_t block, const int32_t* row_ptr,
+                         int32_t row_ptr_stride, const int32_t* col_idx, int64_t max_k, float softmax_scale,
+                         float* lse, cudaStream_t stream) {
+    bsa_status_t st;
+    if ((st = check_tensor(q, "q", B > 1)) || (st = check_tensor(k, "k", B > 1)) || (st = check_tensor(v, "v", B > 1)) ||
+        (st = check_tensor(out, "out", B > 1)))
+        return st;
+    if ((st = attn_common_checks(q, k, v, out, Hq, Hkv, d, block, row_ptr, col_idx, max_k))) return st;
+    if (B < 1 || B > kMaxBatch || N < 1) return fail(BSA_ERR_INVALID_ARG, "bad B=%d / N=%d", B, N);
+    const int nb = (N + block - 1) / block;
+    if (nb > kMaxBlocks) return fail(BSA_ERR_UNSUPPORTED, "at most %d blocks per sequence", kMaxBlocks);
+    if (row_ptr_stride < nb + 1) return fail(BSA_ERR_INVALID_ARG, "row_ptr_stride must be >= nb + 1");
+    if (static_cast<int64_t>(Hkv) * nb * (Hq / Hkv) > 0x7FFFFFFFll) return fail(BSA_ERR_UNSUPPORTED, "grid too large");
+    bsa_status_t est;
+    unsigned* err = device_error_word(&est);
+    if (!err) return est;
+    const int eb = elt_bytes(q.dtype);
+    CUtensorMap tq, tk, tv;
+    if ((st = make_map(&tq, q.ptr, eb, d, N, Hq, B, q.stride_t, q.stride_h, B > 1 ? q.stride_b : q.stride_t * N, 128, "q")) ||
+        (st = make_map(&tk, k.ptr, eb, d, N, Hkv, B, k.stride_t, k.stride_h, B > 1 ? k.stride_b : k.stride_t * N, block, "k")) ||
+        (st = make_map(&tv, v.ptr, eb, d, N, Hkv, B, v.stride_t, v.stride_h, B > 1 ? v.stride_b : v.stride_t * N, block, "v")))
+        return st;
+    AttnArgs a;
+    std::memset(&a, 0, sizeof a);
+    a.B = B;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.d = d;
+    a.block = block;
+    a.nb_max = nb;
+    a.N = N;
+    a.cu_seqlens = nullptr;
+    for (int b = 0; b < B; ++b) a.seqlen[b] = N;
+    a.row_ptr = row_ptr;
+    a.row_ptr_stride = row_ptr_stride;
+    a.col_idx = col_idx;
+    a.max_k = max_k;
+    const float tau = softmax_scale > 0.f ? softmax_scale : 1.f / std::sqrt(static_cast<float>(d));
+    const bool fp8 = q.dtype == BSA_FP8_E4M3;
+    a.scale_log2 = tau * 1.4426950408889634f * (fp8 ? q.scale * k.scale : 1.f);
+    a.out_scale = fp8 ? v.scale : 1.f;
+    a.out = out.ptr;
+    a.osb = out.stride_b;
+    a.ost = out.stride_t;
+    a.osh = out.stride_h;
+    a.lse = lse;
+    a.lse_stride = N;
+    a.err = err;
+    cudaError_t e = launch_attention(fp8, false, tq, tk, tv, a, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "bsa_prefill launch");
+    return BSA_OK;
+}
+
+bsa_status_t bsa_prefill_paged(bsa_tensor_t q, bsa_tensor_t out, const int32_t* cu_seqlens, const int32_t* seqlens_host,
+                               int32_t B, bsa_tensor_t k_cache, bsa_tensor_t v_cache, int32_t num_pages,
+                               int32_t page_size, const int32_t* page_table, int32_t max_pages, int32_t Hq,
+                               int32_t Hkv, int32_t d, int32_t block, const int32_t* row_ptr,
+                               int32_t row_ptr_stride, const int32_t* col_idx, int64_t max_k, float softmax_scale,
+                               float* lse, cudaStream_t stream) {
+    bsa_status_t st;
+    if ((st = check_tensor(q, "q", false)) || (st = check_tensor(out, "out", false)) ||
+        (st = check_tensor(k_cache, "k_cache", true)) || (st = check_tensor(v_cache, "v_cache", true)))
+        return st;
+    if ((st = attn_common_checks(q, k_cache, v_cache, out, Hq, Hkv, d, block, row_ptr, col_idx, max_k))) return st;
+    if (!cu_seqlens || !seqlens_host || !page_table) return fail(BSA_ERR_INVALID_ARG, "null pointer argument");
+    if (B < 1 || B > kMaxBatch) return fail(BSA_ERR_UNSUPPORTED, "B must be in [1, %d]", kMaxBatch);
+    if (page_size != 64 || block % page_size) return fail(BSA_ERR_UNSUPPORTED, "page_size must be 64 and divide block");
+    if (num_pages < 1 || max_pages < 1) return fail(BSA_ERR_INVALID_ARG, "num_pages/max_pages must be positive");
+    AttnArgs a;
+    std::memset(&a, 0, sizeof a);
+    int64_t total = 0;
+    int nb_max = 0, n_max = 0;
+    for (int b = 0; b < B; ++b) {
+        const int n = seqlens_host[b];
+        if (n < 1) return fail(BSA_ERR_INVALID_ARG, "seqlens_host[%d]=%d must be positive", b, n);
+        const int nb = (n + block - 1) / block;
+        if (nb > kMaxBlocks) return fail(BSA_ERR_UNSUPPORTED, "at most %d blocks per sequence", kMaxBlocks);
+        if ((n + page_size - 1) / page_size > max_pages)
+            return fail(BSA_ERR_INVALID_ARG, "sequence %d needs more than max_pages pages", b);
+        a.seqlen[b] = n;
+        total += n;
+        nb_max = nb > nb_max ? nb : nb_max;
+        n_max = n > n_max ? n : n_max;
+    }
+    if (row_ptr_stride < nb_max + 1) return fail(BSA_ERR_INVALID_ARG, "row_ptr_stride must be >= max nb + 1");
+    bsa_status_t est;
+    unsigned* err = device_error_word(&est);
+    if (!err) return est;
+    const int eb = elt_bytes(q.dtype);
+    CUtensorMap tq, tk, tv;
+    if ((st = make_map(&tq, q.ptr, eb, d, total, Hq, 1, q.stride_t, q.stride_h, q.stride_t * total, 128, "q")) ||
+        (st = make_map(&tk, k_cache.ptr, eb, d, page_size, Hkv, num_pages, k_cache.stride_t, k_cache.stride_h,
+                       k_cache.stride_b, 64, "k_cache")) ||
+        (st = make_map(&tv, v_cache.ptr, eb, d, page_size, Hkv, num_pages, v_cache.stride_t, v_cache.stride_h,
+                       v_cache.stride_b, 64, "v_cache")))
+        return st;
+    a.B = B;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.d = d;
+    a.block = block;
+    a.nb_max = nb_max;
+    a.N = n_max;
+    a.cu_seqlens = cu_seqlens;
+    a.row_ptr = row_ptr;
+    a.row_ptr_stride = row_ptr_stride;
+    a.col_idx = col_idx;
+    a.max_k = max_k;
+    a.page_table = page_table;
+    a.max_pages = max_pages;
+    a.page_size = page_size;
+    a.num_pages = num_pages;
+    const float tau = softmax_scale > 0.f ? softmax_scale : 1.f / std::sqrt(static_cast<float>(d));
+    const bool fp8 = q.dtype == BSA_FP8_E4M3;
+    a.scale_log2 = tau * 1.4426950408889634f * (fp8 ? q.scale * k_cache.scale : 1.f);
+    a.out_scale = fp8 ? v_cache.scale : 1.f;
+    a.out = out.ptr;
+    a.osb = 0;
+    a.ost = out.stride_t;
+    a.osh = out.stride_h;
+    a.lse = lse;
+    a.lse_stride = n_max;
+    a.err = err;
+    cudaError_t e = launch_attention(fp8, true, tq, tk, tv, a, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "bsa_prefill_paged launch");
+    return BSA_OK;
+}
+
+const char* bsa_last_error(void) { return g_last_error.c_str(); }
+
+bsa_status_t bsa_check_device_error(cudaStream_t stream) {
+    cudaError_t e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    unsigned v = 0;
+    e = cudaMemcpyFromSymbol(&v, g_device_error, sizeof v);
+    if (e != cudaSuccess) return cuda_fail(e, "read device error word");
+    const unsigned zero = 0;
+    e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof zero);
+    if (e != cudaSuccess) return cuda_fail(e, "clear device error word");
+    if (v & kDevErrTimeout) return fail(BSA_ERR_TIMEOUT, "a kernel wait ran out of time");
+    if (v & kDevErrInvalidList) return fail(BSA_ERR_INVALID_LIST, "a list entry was outside [0, query block]");
+    return BSA_OK;
+}
+
+}  // extern "C"

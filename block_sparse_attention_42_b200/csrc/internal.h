@@ -1,0 +1,68 @@
+// internal.h -- launch interfaces shared between the C-ABI front end (abi.cu) and the kernel
+// translation units.  Not part of the public ABI.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace bsa {
+
+// Device error word bits (read back by bsa_check_device_error).
+constexpr unsigned kDevErrInvalidList = 1u;
+constexpr unsigned kDevErrTimeout = 2u;
+
+constexpr int kMaxBatch = 256;     // sequences per call
+constexpr int kMaxBlocks = 2048;   // query blocks per sequence
+
+struct TensorArg {
+    const void* ptr;
+    int64_t sb, st, sh;  // element strides
+    float scale;
+};
+
+// a1: pooled block representations.  Writes qbar [B,Hq,nb,d], kbar [B,Hkv,nb,d] and
+// vbar [B,Hkv,nb] (fp32).  dtype: 0 bf16, 1 e4m3, 2 fp32.
+cudaError_t launch_pool(int dtype, TensorArg q, TensorArg k, TensorArg v, int B, int N, int Hq, int Hkv, int d,
+                        int block, float* qbar, float* kbar, float* vbar, cudaStream_t s);
+
+// a2: block scores from pooled representations.
+cudaError_t launch_score(const float* qbar, const float* kbar, const float* vbar, int B, int Hq, int Hkv, int nb,
+                         int d, float tau, int metric, float* scores, int nb_stride, cudaStream_t s);
+
+struct SelectSeqs {
+    int32_t B;
+    int32_t nb[kMaxBatch];
+    int64_t kstar[kMaxBatch];
+};
+
+// a3 + a4: TPD budgets into row_ptr, then per-row top-k lists into col_idx.
+cudaError_t launch_select(const float* scores, const SelectSeqs& seqs, int Hq, int nb_stride, bool decay_half,
+                          int32_t* row_ptr, int32_t* col_idx, int64_t max_k, cudaStream_t s);
+
+// a5: block-sparse prefill.
+struct AttnArgs {
+    int B, Hq, Hkv, d, block;
+    int nb_max;                  // max blocks over sequences
+    int N;                       // dense layout: sequence length
+    const int32_t* cu_seqlens;   // paged layout: device prefix offsets (nullptr for dense)
+    int32_t seqlen[kMaxBatch];   // per-sequence lengths (dense: all N)
+    const int32_t* row_ptr;
+    int row_ptr_stride;
+    const int32_t* col_idx;
+    int64_t max_k;
+    const int32_t* page_table;   // paged only
+    int max_pages, page_size, num_pages;
+    float scale_log2;            // softmax scale * log2(e) (* q_scale * k_scale for FP8)
+    float out_scale;             // multiplies the normalised output (v_scale for FP8)
+    void* out;
+    int64_t osb, ost, osh;       // out element strides
+    float* lse;
+    int64_t lse_stride;          // tokens per (b, h) row of lse
+    unsigned* err;
+};
+
+cudaError_t launch_attention(bool fp8, bool paged, const CUtensorMap& tq, const CUtensorMap& tk,
+                             const CUtensorMap& tv, const AttnArgs& a, cudaStream_t s);
+
+}  // namespace bsa

@@ -1,0 +1,144 @@
+/*
+ * bsa.h -- C ABI of the B200 (sm_100a) Stem block-sparse prefill library (libbsa.so).
+ *
+ * The path has three steps, each a call below:
+ *   stem_score   OAM block scoring: pooled per-block Q/K representations and one GEMM,
+ *                weighted by the key block's mean value norm.
+ *                ["腾讯混元Stem稀疏注意力算法：长文推理加速新SOTA" (cn486), §3.2 输出感知度量（OAM）
+ *                 and §二.2.1 Stem算子优化: block-level Q/K representations + one standard GEMM,
+ *                 no softmax, no gather.]
+ *   stem_select  TPD budget generation fused with per-row top-k selection, emitting compact
+ *                ascending KV-block lists per (sequence, query head, query block).
+ *                [same page, §3.1 Token位置衰减策略（TPD） and §二.2.1: budget generation and
+ *                 selection sort fused into one operator.]
+ *   bsa_prefill / bsa_prefill_paged
+ *                block-sparse causal prefill attention that loops only over the prebuilt
+ *                list; a skipped block contributes exactly nothing (all of its scores are
+ *                -inf).  The paged variant reads K/V from a page pool through a page table.
+ *                [same page, §二.2.2 BSA算子优化.]
+ *
+ * Conventions shared by every call:
+ *   - All pointers except those marked "host" are device pointers on the current device.
+ *     The caller owns every buffer; the library allocates no device memory in these calls.
+ *   - Calls are asynchronous on `stream`.  Argument errors are returned synchronously, with
+ *     nothing launched, and the message is available from bsa_last_error().  A failed launch
+ *     returns BSA_ERR_CUDA.  Errors found by kernels while running (an out-of-range list
+ *     entry, an internal wait that ran out of time) are recorded in a per-device error word
+ *     that bsa_check_device_error() reads.
+ *   - Tensors are described by bsa_tensor_t: element strides of batch, token and head; the
+ *     feature (head_dim) dimension is contiguous; the base pointer and every stride must be
+ *     16-byte aligned in bytes.  `scale` is the per-tensor dequantisation scale of FP8 data
+ *     (value = code * scale) and is ignored for BF16/FP32.
+ *   - Supported shapes: head_dim d in {64, 128}; block in {64, 128}; Hq % Hkv == 0;
+ *     query and key lengths are equal (prefill without a prefix); at most 2048 blocks per
+ *     sequence.  FP8 attention requires d = 128.  softmax_scale <= 0 means 1/sqrt(d).
+ */
+#ifndef BSA_H_
+#define BSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    BSA_OK = 0,
+    BSA_ERR_INVALID_ARG = 1,  /* a null pointer, a bad size, stride or alignment */
+    BSA_ERR_UNSUPPORTED = 2,  /* a valid request outside the supported shapes/dtypes */
+    BSA_ERR_CUDA = 3,         /* a CUDA runtime/driver call or a launch failed */
+    BSA_ERR_WORKSPACE = 4,    /* the workspace is missing or too small */
+    BSA_ERR_INVALID_LIST = 5, /* (device) a list entry was outside [0, query block] */
+    BSA_ERR_TIMEOUT = 6       /* (device) an internal pipeline wait ran out of time */
+} bsa_status_t;
+
+typedef enum { BSA_BF16 = 0, BSA_FP8_E4M3 = 1, BSA_FP32 = 2 } bsa_dtype_t;
+
+/* Block metric.  OAM (default): S = tau * Qbar.Kbar + ln(vbar); SAM: S = tau * Qbar.Kbar
+ * (attention score only, the prior-art metric); OAM_MUL: S = tau * Qbar.Kbar * vbar. */
+typedef enum { BSA_METRIC_OAM = 0, BSA_METRIC_SAM = 1, BSA_METRIC_OAM_MUL = 2 } bsa_metric_t;
+
+typedef struct {
+    void* ptr;        /* element [0, 0, 0, 0] */
+    int32_t dtype;    /* bsa_dtype_t */
+    float scale;      /* FP8 dequantisation scale; ignored otherwise */
+    int64_t stride_b; /* elements between batch entries (pages, for a paged cache) */
+    int64_t stride_t; /* elements between tokens (slots, for a paged cache) */
+    int64_t stride_h; /* elements between heads */
+} bsa_tensor_t;
+
+/* TPD budget of one sequence with nb query blocks, computed on the HOST (the same rule the
+ * select kernel runs on the device): k_out[i] (host array of nb) receives the number of KV
+ * blocks kept by query block i; returns their sum K*, or -1 for invalid arguments.
+ * density in (0, 1]; tpd_decay in {0 (uniform), 0.5 (keep ratio ~ (i+1)^-1/2)}.  Use it to
+ * size col_idx (max_k >= K* of every sequence).  [cn486 page, §3.1 TPD.] */
+int64_t bsa_tpd_budget(int32_t nb, double density, double tpd_decay, int32_t* k_out);
+
+/* Bytes of device workspace stem_score needs for B sequences of nb blocks. */
+size_t bsa_score_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int32_t nb, int32_t d);
+
+/* OAM block scores.  q [B, N, Hq, d], k and v [B, N, Hkv, d] (all the same dtype: BF16,
+ * FP8_E4M3 or FP32).  For every (b, query head h, query block i, key block j <= i):
+ *     scores[b, h, i, j] = tau * Qbar[b,h,i] . Kbar[b,h/G,j]  (+ ln vbar[b,h/G,j] for OAM)
+ * with Qbar/Kbar the means of the block's token vectors (dequantised), vbar the mean L2 norm
+ * of the block's value vectors, tau = softmax_scale.  scores is fp32 [B, Hq, nb_stride,
+ * nb_stride] (nb_stride >= nb = ceil(N/block)); entries with j > i inside 64x64 tiles that
+ * touch the diagonal are -inf, tiles wholly above it are not written.  ws: device workspace
+ * of at least bsa_score_workspace_bytes() bytes, 256-byte aligned. */
+bsa_status_t stem_score(bsa_tensor_t q, bsa_tensor_t k, bsa_tensor_t v, int32_t B, int32_t N,
+                        int32_t Hq, int32_t Hkv, int32_t d, int32_t block, int32_t metric,
+                        float softmax_scale, float* scores, int32_t nb_stride, void* ws,
+                        size_t ws_bytes, cudaStream_t stream);
+
+/* TPD budget + per-row top-k.  scores as written by stem_score; nb_per_seq (host, B entries)
+ * gives each sequence's block count (<= nb_stride).  Outputs:
+ *   row_ptr [B, nb_stride + 1] int32: row_ptr[b][i] is the offset of query block i's list
+ *           inside col_idx[b][h][...] (identical for every head of a sequence); entries past
+ *           nb_b repeat the total.
+ *   col_idx [B, Hq, max_k] int32: the list of row (b, h, i) is the sink block 0, the diagonal
+ *           block i and the k_i - 2 highest-scoring blocks among 1..i-1 (NaN counts as -inf,
+ *           equal scores prefer the smaller index), in ascending order.
+ * max_k must be >= the budget total of every sequence (bsa_tpd_budget). */
+bsa_status_t stem_select(const float* scores, int32_t B, int32_t Hq, const int32_t* nb_per_seq,
+                         int32_t nb_stride, double density, double tpd_decay, int32_t* row_ptr,
+                         int32_t* col_idx, int64_t max_k, cudaStream_t stream);
+
+/* Block-sparse causal prefill.  q [B, N, Hq, d]; k, v [B, N, Hkv, d] (BF16, or FP8_E4M3 with
+ * per-tensor scales); out [B, N, Hq, d] BF16.  For token t of head h the allowed keys are the
+ * tokens s <= t whose block is in the list (row_ptr/col_idx as produced by stem_select, with
+ * row_ptr_stride ints per sequence); out = softmax over the allowed keys of
+ * softmax_scale * q.k, times v.  lse (nullable) receives fp32 [B, Hq, N] natural-log
+ * log-sum-exp of the scaled scores. */
+bsa_status_t bsa_prefill(bsa_tensor_t q, bsa_tensor_t k, bsa_tensor_t v, bsa_tensor_t out,
+                         int32_t B, int32_t N, int32_t Hq, int32_t Hkv, int32_t d, int32_t block,
+                         const int32_t* row_ptr, int32_t row_ptr_stride, const int32_t* col_idx,
+                         int64_t max_k, float softmax_scale, float* lse, cudaStream_t stream);
+
+/* Paged-KV variant.  q and out are packed varlen [sum N_b, Hq, d] (stride_b unused);
+ * cu_seqlens (device, B+1) gives each sequence's first token; seqlens_host (host, B) its
+ * length.  k_cache/v_cache are page pools [num_pages, page_size, Hkv, d] described with
+ * stride_b = page stride and stride_t = slot stride; page_table [B, max_pages] int32 maps a
+ * sequence's logical page p (tokens p*page_size ...) to a physical page.  page_size must be
+ * 64 and divide `block`.  Lists and lse ([B, Hq, max_b N_b]) as in bsa_prefill. */
+bsa_status_t bsa_prefill_paged(bsa_tensor_t q, bsa_tensor_t out, const int32_t* cu_seqlens,
+                               const int32_t* seqlens_host, int32_t B, bsa_tensor_t k_cache,
+                               bsa_tensor_t v_cache, int32_t num_pages, int32_t page_size,
+                               const int32_t* page_table, int32_t max_pages, int32_t Hq,
+                               int32_t Hkv, int32_t d, int32_t block, const int32_t* row_ptr,
+                               int32_t row_ptr_stride, const int32_t* col_idx, int64_t max_k,
+                               float softmax_scale, float* lse, cudaStream_t stream);
+
+/* Message of the last error returned on the calling thread ("" if none). */
+const char* bsa_last_error(void);
+
+/* Synchronises `stream`, then reads and clears the current device's error word: returns
+ * BSA_ERR_INVALID_LIST or BSA_ERR_TIMEOUT if a kernel recorded one, else BSA_OK. */
+bsa_status_t bsa_check_device_error(cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BSA_H_ */

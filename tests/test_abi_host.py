@@ -1,0 +1,95 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports every symbol
+include/bsa.h declares, its host TPD budget equals the oracle's bit for bit, and argument
+errors come back as status codes before anything touches the device."""
+import ctypes
+import re
+from pathlib import Path
+
+import numpy as np
+import pytest
+
+ROOT = Path(__file__).resolve().parent.parent
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from block_sparse_attention_42_b200 import binding, build
+    build.build()
+    return binding.lib()
+
+
+def _declared_functions():
+    text = (ROOT / "include" / "bsa.h").read_text()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b([a-z_][a-z0-9_]*)\s*\(", text)) - {"if", "sizeof"})
+
+
+def test_exports_every_declared_symbol(lib):
+    from block_sparse_attention_42_b200 import binding
+    names = _declared_functions()
+    assert set(names) == set(binding.EXPORTS)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_host_budget_equals_oracle_exhaustive(lib, orc):
+    from block_sparse_attention_42_b200 import binding
+    for decay in (0.5, 0.0):
+        for density in (0.1, 0.2, 0.25, 0.5, 0.8, 1.0):
+            for nb in range(1, 2049) if decay == 0.5 and density == 0.25 else range(1, 2049, 37):
+                k, tot = binding.bsa_tpd_budget(nb, density, decay)
+                ko, toto = orc.tpd_budget(nb, density, decay)
+                assert tot == toto and np.array_equal(k.numpy(), ko), (nb, density, decay)
+
+
+def test_host_budget_rejects_bad_args(lib):
+    k = (ctypes.c_int32 * 8)()
+    assert lib.bsa_tpd_budget(0, 0.5, 0.5, k) == -1
+    assert lib.bsa_tpd_budget(8, 0.0, 0.5, k) == -1
+    assert lib.bsa_tpd_budget(8, 0.5, 0.25, k) == -1
+
+
+def _t(ptr=0x10000, dtype=0, st=1024, sh=128, sb=1 << 20, scale=1.0):
+    from block_sparse_attention_42_b200.binding import BsaTensor
+    return BsaTensor(ptr, dtype, scale, sb, st, sh)
+
+
+def test_argument_errors_return_status(lib):
+    P = ctypes.c_void_p
+    ws = P(0x20000)
+    sc = P(0x30000)
+    # null q
+    assert lib.stem_score(_t(ptr=0), _t(), _t(), 1, 1024, 8, 8, 128, 128, 0, 0.0, sc, 8, ws, 1 << 30, None) == 1
+    # misaligned base pointer
+    assert lib.stem_score(_t(ptr=0x10008), _t(), _t(), 1, 1024, 8, 8, 128, 128, 0, 0.0, sc, 8, ws, 1 << 30, None) == 1
+    # stride not a multiple of 16 bytes
+    assert lib.stem_score(_t(st=1023), _t(), _t(), 1, 1024, 8, 8, 128, 128, 0, 0.0, sc, 8, ws, 1 << 30, None) == 1
+    # Hq % Hkv != 0
+    assert lib.stem_score(_t(), _t(), _t(), 1, 1024, 6, 4, 128, 128, 0, 0.0, sc, 8, ws, 1 << 30, None) == 1
+    # unsupported head_dim / block
+    assert lib.stem_score(_t(), _t(), _t(), 1, 1024, 8, 8, 96, 128, 0, 0.0, sc, 8, ws, 1 << 30, None) == 2
+    assert lib.stem_score(_t(), _t(), _t(), 1, 1024, 8, 8, 128, 32, 0, 0.0, sc, 8, ws, 1 << 30, None) == 2
+    # workspace too small
+    assert lib.stem_score(_t(), _t(), _t(), 1, 1024, 8, 8, 128, 128, 0, 0.0, sc, 8, ws, 16, None) == 4
+    # nb_stride too small
+    assert lib.stem_score(_t(), _t(), _t(), 1, 1024, 8, 8, 128, 128, 0, 0.0, sc, 4, ws, 1 << 30, None) == 1
+    nbp = (ctypes.c_int32 * 1)(8)
+    # density out of range, decay unsupported, max_k too small
+    assert lib.stem_select(sc, 1, 8, nbp, 8, 0.0, 0.5, P(0x40000), P(0x50000), 100, None) == 1
+    assert lib.stem_select(sc, 1, 8, nbp, 8, 0.5, 0.3, P(0x40000), P(0x50000), 100, None) == 2
+    assert lib.stem_select(sc, 1, 8, nbp, 8, 0.5, 0.5, P(0x40000), P(0x50000), 3, None) == 1
+    # attention: FP8 needs d=128/block=128; out must be BF16; null lists
+    f8 = dict(dtype=1, scale=0.5)
+    assert lib.bsa_prefill(_t(**f8), _t(**f8), _t(**f8), _t(), 1, 1024, 8, 8, 64, 128, P(1), 9, P(1), 36, 0.0,
+                           None, None) == 2
+    assert lib.bsa_prefill(_t(), _t(), _t(), _t(dtype=2), 1, 1024, 8, 8, 128, 128, P(1), 9, P(1), 36, 0.0,
+                           None, None) == 2
+    assert lib.bsa_prefill(_t(), _t(), _t(), _t(), 1, 1024, 8, 8, 128, 128, None, 9, P(1), 36, 0.0, None, None) == 1
+    # FP8 with a non-positive scale
+    assert lib.bsa_prefill(_t(dtype=1, scale=0.0), _t(**f8), _t(**f8), _t(), 1, 1024, 8, 8, 128, 128, P(1), 9,
+                           P(1), 36, 0.0, None, None) == 1
+    # paged: page size must be 64
+    sl = (ctypes.c_int32 * 1)(1024)
+    assert lib.bsa_prefill_paged(_t(), _t(), P(1), sl, 1, _t(), _t(), 100, 32, P(1), 16, 8, 8, 128, 128, P(1), 9,
+                                 P(1), 36, 0.0, None, None) == 2
+    assert lib.bsa_last_error().decode() != ""
