@@ -128,6 +128,19 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def reduce_max(x: float, world: int, device) -> float:
+    """Max over ranks of a per-rank timing (the only collective: not on the data path)."""
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(eff_flop_per_rank: float, world: int, ms_per_step: float) -> float:
+    """Weak scaling: every rank runs its own problem of the same size."""
+    return eff_flop_per_rank * world / (ms_per_step * 1e-3) / 1e12
+
+
 def peaks():
     p = ROOT / "MEASURED_PEAKS.json"
     if p.exists():
@@ -198,10 +211,7 @@ def run_ours(args, rank, world, device):
     total_ms = ev[0].elapsed_time(ev[1])
     select_ms = [per[s][0].elapsed_time(per[s][1]) for s in range(args.steps)]
     attn_ms = [per[s][1].elapsed_time(per[s][2]) for s in range(args.steps)]
-    t = torch.tensor([total_ms], dtype=torch.float64, device=device)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    max_ms = float(t.item())
+    max_ms = reduce_max(total_ms, world, device)
     bsa.bsa_check_device_error(device)
 
     res = dict(total_ms=max_ms, ms_per_step=max_ms / args.steps, eff_flop=eff,
@@ -255,10 +265,7 @@ def run_ours(args, rank, world, device):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize(device)
-        t = torch.tensor([e0.elapsed_time(e1) / n_e2e], dtype=torch.float64, device=device)
-        if world > 1:
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        res["e2e_ms"] = float(t.item())
+        res["e2e_ms"] = reduce_max(e0.elapsed_time(e1) / n_e2e, world, device)
         res["h2d_bytes"] = sum(x.numel() * x.element_size() for x in (q, k, v))
         res["d2h_bytes"] = out.numel() * out.element_size()
         del hq, hk, hv, hout, dq, dk, dv
@@ -404,7 +411,7 @@ def main():
         fp8 = res["fp8"]
         peak = (pk.get("bf16_tflops_sustained", pk["bf16_tflops"]) * (2.0 if fp8 else 1.0))
         attn_ach = res["eff_flop"] / (res["attn_ms_mean"] * 1e-3) / 1e12
-        value = res["eff_flop"] * world / (res["ms_per_step"] * 1e-3) / 1e12
+        value = whole_job_tflops(res["eff_flop"], world, res["ms_per_step"])
         w = res["w"]
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -431,7 +438,7 @@ def main():
             line["ideal_line_ratio"] = res["attn_ms_mean"] / (res["dense_ms"] * rho_eff)
             line["rho_eff"] = rho_eff
         if "e2e_ms" in res:
-            line["e2e"] = {"value": res["eff_flop"] * world / (res["e2e_ms"] * 1e-3) / 1e12, "unit": "TFLOP/s",
+            line["e2e"] = {"value": whole_job_tflops(res["eff_flop"], world, res["e2e_ms"]), "unit": "TFLOP/s",
                            "h2d_bytes_per_step": res["h2d_bytes"], "d2h_bytes_per_step": res["d2h_bytes"],
                            "ms_per_step": res["e2e_ms"]}
         if res["cpu"] is not None:

@@ -9,7 +9,8 @@ import torch
 
 # Tolerances (also written in the design doc):
 SCORE_REL = 1e-5          # scores: |gpu - oracle| <= 1e-5 * max(|oracle|, condition scale)
-BF16_MAX_ABS = 2e-2       # BF16 attention output
+BF16_MAX_ABS = 2e-2       # BF16 attention output: |g - o| <= 2e-2 + BF16_ULP_REL * |o|
+BF16_ULP_REL = 4 * 2.0 ** -9   # four BF16 half-ulps: output rounding + P rounding + accumulation
 BF16_REL_L2 = 1e-2
 FP8_REL_L2 = 5e-2         # FP8 attention output
 LSE_ABS = 1e-3            # natural-log LSE (fp32 log2/ex2 approximations, bf16-free)
@@ -52,6 +53,16 @@ def assert_scores_close(gpu, ora, scale, nb):
     lim = (SCORE_REL * np.maximum(np.abs(o), scale[..., :nb, :nb]))[fin] + 1e-30
     worst = float(np.max(err / lim)) if err.size else 0.0
     assert worst <= 1.0, f"score error {worst:.3f} x tolerance"
+
+
+def assert_bf16_close(got, ref):
+    """Elementwise |got - ref| <= 2e-2 + 4 * 2^-9 |ref| (absolute for unit-scale outputs, BF16
+    half-ulps for large ones) and rel-L2 <= 1e-2."""
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    excess = np.abs(got - ref) - (BF16_MAX_ABS + BF16_ULP_REL * np.abs(ref))
+    assert np.all(excess <= 0), f"max-abs bound exceeded by {float(np.max(excess)):.3e}"
+    assert rel_l2(got, ref) <= BF16_REL_L2, rel_l2(got, ref)
 
 
 def rel_l2(a, b):

@@ -168,8 +168,7 @@ def test_attention_bf16_matches_oracle(orc, name, w, N, storage, full):
     rows = H.all_rows(B, Hq, N) if full else H.sample_rows(B, Hq, N, w.block)
     ref, ref_lse = H.oracle_attention(orc, q, k, v, w.block, rp, ci, H.default_tau(d), rows)
     got = H.gather_rows(out, rows)
-    assert np.max(np.abs(got - ref)) <= H.BF16_MAX_ABS
-    assert H.rel_l2(got, ref) <= H.BF16_REL_L2
+    H.assert_bf16_close(got, ref)
     got_lse = np.array([lse[b, h, t].item() for b, h, t in rows]) if not full else \
         lse.permute(0, 1, 2).cpu().numpy().reshape(-1)
     assert np.max(np.abs(got_lse - ref_lse)) <= H.LSE_ABS
@@ -198,31 +197,27 @@ def test_density_one_is_dense_causal(orc):
     ref = torch.nn.functional.scaled_dot_product_attention(
         q.double().transpose(1, 2), k.double().repeat_interleave(G, 2).transpose(1, 2),
         v.double().repeat_interleave(G, 2).transpose(1, 2), is_causal=True).transpose(1, 2)
-    err = (out.double() - ref).abs().max().item()
-    assert err <= H.BF16_MAX_ABS
-    assert H.rel_l2(out.double().cpu(), ref.cpu()) <= H.BF16_REL_L2
+    H.assert_bf16_close(out.double().cpu().numpy(), ref.cpu().numpy())
 
 
 def test_skipped_blocks_do_not_matter():
-    """K/V of blocks outside every list may hold anything (1e4, NaN): the output is bit-identical."""
-    w = inputs.Workload("skip", 1, 2, 1, 1024, 128, 128, "bf16", 0.2, "normal", 16)
+    """K/V of blocks outside query block i's list may hold anything (1e4, NaN): the outputs of
+    block i's rows are bit-identical."""
+    w = inputs.Workload("skip", 1, 1, 1, 1024, 128, 128, "bf16", 0.2, "normal", 16)
     q, k, v, *_ = _inputs(w)
     rp, ci = _lists(q, k, v, w.block, 0.2)
     out1 = bsa.bsa_prefill(q, k, v, w.block, rp, ci)
-    nb = 8
-    used = set()
-    cpu_rp, cpu_ci = rp.cpu().numpy(), ci.cpu().numpy()
-    for h in range(w.Hq):
-        used |= set(cpu_ci[0, h, : cpu_rp[0, nb]].tolist())
+    i = 7
+    kept = set(ci[0, 0, rp[0, i]:rp[0, i + 1]].cpu().tolist())
+    assert len(kept) < i + 1
     k2, v2 = k.clone(), v.clone()
-    for j in range(nb):
-        if j not in used:
+    for j in range(i + 1):
+        if j not in kept:
             k2[:, j * 128:(j + 1) * 128] = 1e4
             v2[:, j * 128:(j + 1) * 128] = float("nan")
-    assert len(used) < nb
     out2 = bsa.bsa_prefill(q, k2, v2, w.block, rp, ci)
     torch.cuda.synchronize()
-    assert torch.equal(out1, out2)
+    assert torch.equal(out1[:, i * 128:(i + 1) * 128], out2[:, i * 128:(i + 1) * 128])
 
 
 def test_paged_equals_contiguous():
