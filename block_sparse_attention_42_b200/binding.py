@@ -23,7 +23,7 @@ STATUS = {0: "BSA_OK", 1: "BSA_ERR_INVALID_ARG", 2: "BSA_ERR_UNSUPPORTED", 3: "B
 
 # Every symbol include/bsa.h declares.
 EXPORTS = ["bsa_tpd_budget", "bsa_score_workspace_bytes", "stem_score", "stem_select", "bsa_prefill",
-           "bsa_prefill_paged", "bsa_last_error", "bsa_check_device_error"]
+           "bsa_prefill_paged", "bsa_last_error", "bsa_check_device_error", "stem_score_noalloc"]
 
 
 class BsaError(RuntimeError):
@@ -52,13 +52,14 @@ def lib():
     L.bsa_score_workspace_bytes.argtypes = [i32, i32, i32, i32, i32]
     L.bsa_score_workspace_bytes.restype = ctypes.c_size_t
     L.stem_score.argtypes = [T, T, T, i32, i32, i32, i32, i32, i32, i32, f32, P, i32, P, ctypes.c_size_t, P]
+    L.stem_score_noalloc.argtypes = [T, T, T, i32, i32, i32, i32, i32, i32, i32, f32, P, i32, P]
     L.stem_select.argtypes = [P, i32, i32, P, i32, f64, f64, P, P, i64, P]
     L.bsa_prefill.argtypes = [T, T, T, T, i32, i32, i32, i32, i32, i32, P, i32, P, i64, f32, P, P]
     L.bsa_prefill_paged.argtypes = [T, T, P, P, i32, T, T, i32, i32, P, i32, i32, i32, i32, i32, P, i32, P, i64,
                                     f32, P, P]
     L.bsa_last_error.restype = ctypes.c_char_p
     L.bsa_check_device_error.argtypes = [P]
-    for name in ["stem_score", "stem_select", "bsa_prefill", "bsa_prefill_paged", "bsa_check_device_error"]:
+    for name in ["stem_score", "stem_score_noalloc", "stem_select", "bsa_prefill", "bsa_prefill_paged", "bsa_check_device_error"]:
         getattr(L, name).restype = ctypes.c_int
     _lib = L
     return L
@@ -124,6 +125,22 @@ def stem_score(q, k, v, block: int, metric: int = BSA_METRIC_OAM, softmax_scale:
     st = lib().stem_score(tensor_arg(q, q_scale), tensor_arg(k, k_scale), tensor_arg(v, v_scale), B, N, Hq, Hkv, d,
                           block, metric, float(softmax_scale), _ptr(scores), nbs, _ptr(workspace),
                           workspace.numel(), _stream(q))
+    _check(st)
+    return scores
+
+
+def stem_score_noalloc(q, k, v, block: int, metric: int = BSA_METRIC_OAM, softmax_scale: float = 0.0,
+                       scores=None, nb_stride: int | None = None, q_scale=1.0, k_scale=1.0, v_scale=1.0):
+    """stem_score with the library's fixed 16 MiB scratch instead of a workspace (for callers
+    that cannot allocate device memory).  Calls that overlap on the GPU race on that scratch."""
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    nb = (N + block - 1) // block
+    nbs = nb if nb_stride is None else nb_stride
+    if scores is None:
+        scores = torch.empty(B, Hq, nbs, nbs, dtype=torch.float32, device=q.device)
+    st = lib().stem_score_noalloc(tensor_arg(q, q_scale), tensor_arg(k, k_scale), tensor_arg(v, v_scale), B, N,
+                                  Hq, Hkv, d, block, metric, float(softmax_scale), _ptr(scores), nbs, _stream(q))
     _check(st)
     return scores
 

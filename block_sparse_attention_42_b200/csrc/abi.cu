@@ -159,6 +159,9 @@ bsa_status_t attn_common_checks(const bsa_tensor_t& q, const bsa_tensor_t& k, co
 }
 
 }  // namespace
+
+void set_last_error(const char* msg) { g_last_error = msg; }
+
 }  // namespace bsa
 
 using namespace bsa;

@@ -62,6 +62,9 @@ struct AttnArgs {
     unsigned* err;
 };
 
+// Sets the message bsa_last_error() returns on this thread.
+void set_last_error(const char* msg);
+
 cudaError_t launch_attention(bool fp8, bool paged, const CUtensorMap& tq, const CUtensorMap& tk,
                              const CUtensorMap& tv, const AttnArgs& a, cudaStream_t s);
 

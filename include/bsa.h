@@ -130,6 +130,30 @@ bsa_status_t bsa_prefill_paged(bsa_tensor_t q, bsa_tensor_t out, const int32_t* 
                                int32_t row_ptr_stride, const int32_t* col_idx, int64_t max_k,
                                float softmax_scale, float* lse, cudaStream_t stream);
 
+/* stem_score without a workspace argument, for callers that cannot allocate device memory:
+ * for example a plain C host program that links only this library and has no device
+ * allocator of its own, or a serving runtime whose memory pool owns all of HBM and does not
+ * let a library call cudaMalloc (which would also synchronise the device mid-stream).  It
+ * has no counterpart on the Stem pages; it is a deployment convenience.
+ *
+ * Arguments, layouts, results and errors are those of stem_score.  The pooled Q/K
+ * representations and value norms that stem_score keeps in `ws` live instead in a fixed
+ * 16 MiB array inside the library, which every GPU that loads the library holds until the
+ * process exits.  Problems that need more than that (bsa_score_workspace_bytes() > 16 MiB,
+ * e.g. beyond about 58K tokens at 64 query / 8 KV heads, d = 128, block 128) are rejected
+ * with BSA_ERR_UNSUPPORTED and a message naming both sizes; nothing is launched.  The call
+ * itself allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
+ *   - The first call on each device looks up the array's device address (with that device
+ *     current) and caches it; make that first call before any stream capture.
+ *   - All calls share the one array and it keeps the last call's contents.  Nothing in it has
+ *     to start at zero: every call rewrites all of the scratch it reads.  Calls whose work
+ *     overlaps on the GPU (other streams, or other host threads on the same device) race on
+ *     the array and must be serialised by the caller. */
+bsa_status_t stem_score_noalloc(bsa_tensor_t q, bsa_tensor_t k, bsa_tensor_t v, int32_t B, int32_t N,
+                                int32_t Hq, int32_t Hkv, int32_t d, int32_t block, int32_t metric,
+                                float softmax_scale, float* scores, int32_t nb_stride,
+                                cudaStream_t stream);
+
 /* Message of the last error returned on the calling thread ("" if none). */
 const char* bsa_last_error(void);
 

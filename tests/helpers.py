@@ -49,7 +49,7 @@ def assert_scores_close(gpu, ora, scale, nb):
     fin = np.isfinite(o) & tri
     assert np.array_equal(np.isfinite(g) & tri, fin), "finite pattern differs"
     assert np.all(np.isneginf(g[np.isneginf(o) & tri])), "-inf entries differ"
-    err = np.abs(g - o)[fin]
+    err = np.abs(g[fin] - o[fin])
     lim = (SCORE_REL * np.maximum(np.abs(o), scale[..., :nb, :nb]))[fin] + 1e-30
     worst = float(np.max(err / lim)) if err.size else 0.0
     assert worst <= 1.0, f"score error {worst:.3f} x tolerance"
