@@ -4,6 +4,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <string>
@@ -139,6 +140,15 @@ bsa_status_t make_map(CUtensorMap* m, const void* base, int eb, uint64_t d, uint
 }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Attention kernel: the persistent warp-specialised one unless BSA_ATTN_VARIANT=serial selects
+// the one-tile-per-CTA kernel (both compute the same result; tests cross-check them).
+cudaError_t launch_attn(bool fp8, bool paged, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                        const AttnArgs& a, cudaStream_t s) {
+    const char* v = std::getenv("BSA_ATTN_VARIANT");
+    if (v && std::strcmp(v, "serial") == 0) return launch_attention(fp8, paged, tq, tk, tv, a, s);
+    return launch_attention_ws(fp8, paged, tq, tk, tv, a, s);
+}
 
 bsa_status_t attn_common_checks(const bsa_tensor_t& q, const bsa_tensor_t& k, const bsa_tensor_t& v,
                                 const bsa_tensor_t& out, int32_t Hq, int32_t Hkv, int32_t d, int32_t block,
@@ -335,7 +345,7 @@ bsa_status_t bsa_prefill(bsa_tensor_t q, bsa_tensor_t k, bsa_tensor_t v, bsa_ten
     a.lse = lse;
     a.lse_stride = N;
     a.err = err;
-    cudaError_t e = launch_attention(fp8, false, tq, tk, tv, a, stream);
+    cudaError_t e = launch_attn(fp8, false, tq, tk, tv, a, stream);
     if (e != cudaSuccess) return cuda_fail(e, "bsa_prefill launch");
     return BSA_OK;
 }
@@ -410,7 +420,7 @@ bsa_status_t bsa_prefill_paged(bsa_tensor_t q, bsa_tensor_t out, const int32_t* 
     a.lse = lse;
     a.lse_stride = n_max;
     a.err = err;
-    cudaError_t e = launch_attention(fp8, true, tq, tk, tv, a, stream);
+    cudaError_t e = launch_attn(fp8, true, tq, tk, tv, a, stream);
     if (e != cudaSuccess) return cuda_fail(e, "bsa_prefill_paged launch");
     return BSA_OK;
 }

@@ -65,7 +65,12 @@ struct AttnArgs {
 // Sets the message bsa_last_error() returns on this thread.
 void set_last_error(const char* msg);
 
+// One query tile per CTA, serial load -> S -> softmax -> PV per kept block (attn.cu).
 cudaError_t launch_attention(bool fp8, bool paged, const CUtensorMap& tq, const CUtensorMap& tk,
                              const CUtensorMap& tv, const AttnArgs& a, cudaStream_t s);
+// Persistent, warp-specialised: TMA producer, MMA issuer, two softmax warpgroups over two
+// query tiles in flight (attn_ws.cu).  The default.
+cudaError_t launch_attention_ws(bool fp8, bool paged, const CUtensorMap& tq, const CUtensorMap& tk,
+                                const CUtensorMap& tv, const AttnArgs& a, cudaStream_t s);
 
 }  // namespace bsa

@@ -75,8 +75,13 @@ def paged_varlen(density=0.25, seqlens=(16384, 32768, 65536, 131072)) -> Workloa
                     "stem", 4, seqlens=seqlens, page_size=64)
 
 
+def fp8_32k(density=0.25) -> Workload:
+    """The FP8 workload at 32K tokens: a profiling case that still exceeds L2 (Q is 268 MB)."""
+    return Workload("fp8-32k", 1, 64, 8, 32768, 128, 128, "fp8", density, "stem", 3)
+
+
 WORKLOADS = {"tiny-1k": tiny, "gqa-8k": gqa_8k, "sweep-32k": sweep_32k, "fp8-128k": fp8_128k,
-             "paged-varlen": paged_varlen}
+             "paged-varlen": paged_varlen, "fp8-32k": fp8_32k}
 
 
 def _gen(device, seed):
