@@ -1,0 +1,79 @@
+// attn_tiles.cuh -- the work-tile schedule shared by the attention kernels: tile index ->
+// (sequence, KV head, query block, query head), the tile's kept-block list, and the static
+// per-worker walk over tiles.
+#pragma once
+
+#include "internal.h"
+
+namespace bsa {
+
+// Work tile t -> (b, hk, i, g); tiles are ordered sequence-major, then KV head, then query
+// block from the last one down, then the G query heads of the group.
+struct Tile {
+    int b, h, hk, i, n_tok, nb, n_list, l_begin;
+    bool valid;
+};
+
+__device__ __forceinline__ Tile decode_tile(const AttnArgs& a, int t) {
+    Tile T;
+    const int G = a.Hq / a.Hkv;
+    const int per_b = a.Hkv * a.nb_max * G;
+    T.b = t / per_b;
+    int x = t % per_b;
+    const int g = x % G;
+    x /= G;
+    T.i = a.nb_max - 1 - (x % a.nb_max);
+    T.hk = x / a.nb_max;
+    T.h = T.hk * G + g;
+    T.n_tok = a.seqlen[T.b];
+    T.nb = (T.n_tok + a.block - 1) / a.block;
+    T.valid = T.i < T.nb;
+    T.n_list = 0;
+    T.l_begin = 0;
+    if (T.valid) {
+        const int32_t* rp = a.row_ptr + static_cast<int64_t>(T.b) * a.row_ptr_stride;
+        T.l_begin = __ldg(rp + T.i);
+        T.n_list = __ldg(rp + T.i + 1) - T.l_begin;
+        if (T.n_list < 1 || T.n_list > kMaxBlocks || T.l_begin < 0 ||
+            T.l_begin + static_cast<int64_t>(T.n_list) > a.max_k) {
+            T.n_list = 0;  // corrupt row pointer: the tile is skipped
+        }
+    }
+    return T;
+}
+
+// List entry n of the tile; -1 if out of [0, i] (skipped block: scores all -inf).
+__device__ __forceinline__ int list_entry(const AttnArgs& a, const Tile& T, int n) {
+    const int j = __ldg(a.col_idx + (static_cast<int64_t>(T.b) * a.Hq + T.h) * a.max_k + T.l_begin + n);
+    return (j >= 0 && j <= T.i) ? j : -1;
+}
+
+// The static tile sequence of one slot: tiles base + s, base + s + stride, ... that are
+// non-empty.  Every role walks the same sequence.
+struct TileIter {
+    int round, s, base, stride, total;
+    bool active;
+    Tile T;
+    __device__ void init(int s_, int base_, int stride_, int total_) {
+        s = s_;
+        base = base_;
+        stride = stride_;
+        total = total_;
+        round = 0;
+        active = true;
+    }
+    __device__ void next(const AttnArgs& a) {
+        while (true) {
+            const int t = base + s + round * stride;
+            ++round;
+            if (t >= total) {
+                active = false;
+                return;
+            }
+            T = decode_tile(a, t);
+            if (T.valid && T.n_list > 0) return;
+        }
+    }
+};
+
+}  // namespace bsa

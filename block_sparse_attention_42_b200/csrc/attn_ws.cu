@@ -4,20 +4,21 @@
 //  compute run as a pipeline; the KV-block list is built before the inner loop, which then
 //  visits only valid blocks with the dense-attention body; skipped blocks are -inf.]
 //
-// One CTA per SM, 12 warps:
-//   warp 0      TMA producer: Q tiles and a ring of K/V stages, in exactly the order the MMA
-//               warp consumes them
-//   warp 1      MMA issuer (and TMEM owner): S_s = Q_s K^T and O_s += P_s V for two query
-//               tiles ("slots" s = 0, 1) in flight at once, so the tensor cores work on one
-//               slot while the other slot's softmax runs
+// One CTA per SM, 12 warps, two query tiles ("slots" s = 0, 1) in flight:
+//   warp 0      TMA producer: per slot, its Q tile and a private ring of K/V stages
+//   warp 1      MMA issuer (and TMEM owner): S_s = Q_s K^T, then O_s += P_s V with P_s read
+//               from tensor memory (it overwrites S_s in place)
 //   warps 4-7   softmax of slot 0, warps 8-11 softmax of slot 1: one query row per thread;
-//               tcgen05.ld S, online max/sum, P -> shared memory, O rescale in TMEM when the
-//               row max moved, and the tile epilogue (O / l -> BF16, LSE)
-// TMEM (512 columns): S_0 | S_1 | O_0 | O_1, 128 columns each.
+//               tcgen05.ld S, online max/sum, P -> TMEM (BF16 or E4M3), O rescale in TMEM when
+//               the row max grew enough, and the tile epilogue (O / l -> BF16, LSE)
+// The producer and the MMA warp poll both slots and serve whichever is ready, so the two
+// slots run independently and one slot's softmax overlaps the other slot's MMAs.
+// TMEM (512 columns): S_0/P_0 | S_1/P_1 | O_0 | O_1, 128 columns each.
 // Each slot walks its own static sequence of work tiles (tile = query block i of head h), in
 // KV-head-major order with the longest lists first.
 #include <cuda_bf16.h>
 
+#include "attn_tiles.cuh"
 #include "internal.h"
 #include "sm100.cuh"
 
@@ -28,6 +29,18 @@ constexpr int kBM = 128;
 constexpr int kWarps = 12;
 constexpr int kThreads = kWarps * 32;
 constexpr int kSmemLimit = 232448;  // 227 KB of dynamic shared memory per CTA
+constexpr int kMaxStages = 6;       // K/V stages per slot
+constexpr int kListChunk = 128;     // list entries the producer stages in shared memory per slot
+// Polling loops give up after this many SM cycles without progress (about 2 s).
+constexpr long long kPollLimitCycles = 4000000000ll;
+// Register split.  The kernel is launched with 168 registers per thread (384 x 168 = 64512; the
+// build refuses an attn_ws_kernel compiled at any other count).  Warpgroup 0 (producer, MMA,
+// two idle warps) then gives registers back and the two softmax warpgroups take them:
+// 128 x 56 + 256 x 224 = 64512, exactly the launch pool.
+constexpr int kRegsLaunch = 168;
+constexpr int kRegsLow = 56;
+constexpr int kRegsHigh = 224;
+static_assert(128 * kRegsLow + 256 * kRegsHigh <= kThreads * kRegsLaunch, "register split exceeds the launch pool");
 
 template <bool FP8, int D, int BN>
 struct WsCfg {
@@ -36,19 +49,16 @@ struct WsCfg {
     static constexpr int QP = D * EB / 128;
     static constexpr int Q_BYTES = kBM * D * EB;
     static constexpr int KV_BYTES = BN * D * EB;
-    static constexpr int P_BYTES = kBM * BN * EB;
-    static constexpr int FIXED = 2 * Q_BYTES + 2 * P_BYTES;
-    static constexpr int NS_FIT = (kSmemLimit - 2048 - FIXED) / KV_BYTES;
-    static constexpr int NS = NS_FIT > 8 ? 8 : NS_FIT;  // K/V ring stages
+    static constexpr int NSS_FIT = (kSmemLimit - 5120 - 2 * Q_BYTES) / (2 * KV_BYTES);
+    static constexpr int NSS = NSS_FIT > kMaxStages ? kMaxStages : NSS_FIT;  // stages per slot
     static constexpr int OFF_Q = 0;
-    static constexpr int OFF_P = OFF_Q + 2 * Q_BYTES;
-    static constexpr int OFF_RING = OFF_P + 2 * P_BYTES;
-    static constexpr int OFF_BAR = OFF_RING + NS * KV_BYTES;
-    static constexpr int SMEM = OFF_BAR + 1024 + 1024;  // barriers + alignment slack
+    static constexpr int OFF_RING = 2 * Q_BYTES;
+    static constexpr int OFF_BAR = OFF_RING + 2 * NSS * KV_BYTES;
+    static constexpr int SMEM = OFF_BAR + 2048 + 1024;  // barriers, list buffers + alignment slack
     static constexpr int KSTEPS_S = D * EB / 32;
     static constexpr int KSTEPS_O = BN * EB / 32;
     static constexpr int ROWS_PER_KSTEP = 32 / EB;
-    static_assert(NS >= 2, "K/V ring needs at least two stages");
+    static_assert(NSS >= 2, "each slot needs at least two K/V stages");
     static_assert(SMEM <= kSmemLimit, "shared memory budget");
 };
 
@@ -61,81 +71,15 @@ template <bool FP8>
 constexpr float kPScaleLog2 = FP8 ? 5.f : 0.f;
 
 struct Bars {
-    uint64_t kv_full[8], kv_empty[8];
+    uint64_t kv_full[2][kMaxStages], kv_empty[2][kMaxStages];
     uint64_t q_full[2], q_empty[2];
     uint64_t s_full[2], p_full[2], o_done[2];
-    uint64_t drain;
+    uint64_t drain, tmem_free;
     uint32_t tmem_slot;
     int abort_flag;
+    int lst[2][kListChunk];  // producer's staged list entries per slot
 };
-
-// Work tile t -> (b, hk, i, g); tiles are ordered sequence-major, then KV head, then query
-// block from the last one down, then the G query heads of the group.
-struct Tile {
-    int b, h, hk, i, n_tok, nb, n_list, l_begin;
-    bool valid;
-};
-
-__device__ __forceinline__ Tile decode_tile(const AttnArgs& a, int t) {
-    Tile T;
-    const int G = a.Hq / a.Hkv;
-    const int per_b = a.Hkv * a.nb_max * G;
-    T.b = t / per_b;
-    int x = t % per_b;
-    const int g = x % G;
-    x /= G;
-    T.i = a.nb_max - 1 - (x % a.nb_max);
-    T.hk = x / a.nb_max;
-    T.h = T.hk * G + g;
-    T.n_tok = a.seqlen[T.b];
-    T.nb = (T.n_tok + a.block - 1) / a.block;
-    T.valid = T.i < T.nb;
-    T.n_list = 0;
-    T.l_begin = 0;
-    if (T.valid) {
-        const int32_t* rp = a.row_ptr + static_cast<int64_t>(T.b) * a.row_ptr_stride;
-        T.l_begin = rp[T.i];
-        T.n_list = rp[T.i + 1] - T.l_begin;
-        if (T.n_list < 1 || T.n_list > kMaxBlocks || T.l_begin < 0 ||
-            T.l_begin + static_cast<int64_t>(T.n_list) > a.max_k) {
-            T.n_list = 0;  // corrupt row pointer: the tile is skipped (and flagged by the producer)
-        }
-    }
-    return T;
-}
-
-// List entry n of the tile; -1 if out of [0, i] (skipped block: scores all -inf).
-__device__ __forceinline__ int list_entry(const AttnArgs& a, const Tile& T, int n) {
-    const int j = __ldg(a.col_idx + (static_cast<int64_t>(T.b) * a.Hq + T.h) * a.max_k + T.l_begin + n);
-    return (j >= 0 && j <= T.i) ? j : -1;
-}
-
-// Both the producer and the MMA warp run this same event sequence, so ring stages are
-// filled and consumed in the same order.  Per slot: Q load, S(0), then PV(k), S(k+1) ...
-struct Sched {
-    int tile[2], n[2], a[2], round[2];
-    bool active[2];
-    int total, stride, base;
-    __device__ void start(const AttnArgs& aa, int s) {
-        // next non-empty tile of slot s
-        while (true) {
-            const int t = base + s + round[s] * stride;
-            round[s]++;
-            if (t >= total) {
-                active[s] = false;
-                return;
-            }
-            Tile T = decode_tile(aa, t);
-            if (T.valid && T.n_list > 0) {
-                tile[s] = t;
-                n[s] = T.n_list;
-                a[s] = 0;
-                active[s] = true;
-                return;
-            }
-        }
-    }
-};
+static_assert(sizeof(Bars) <= 2048, "barrier region");
 
 template <bool FP8, int D, int BN, bool PAGED>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -147,13 +91,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     Bars* bars = reinterpret_cast<Bars*>(smem + C::OFF_BAR);
     volatile int* abort_flag = &bars->abort_flag;
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int stride = 2 * gridDim.x, base = 2 * blockIdx.x;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < C::NS; ++s) {
-            mbar_init(&bars->kv_full[s], 1);
-            mbar_init(&bars->kv_empty[s], 1);
-        }
         for (int s = 0; s < 2; ++s) {
+            for (int t = 0; t < C::NSS; ++t) {
+                mbar_init(&bars->kv_full[s][t], 1);
+                mbar_init(&bars->kv_empty[s][t], 1);
+            }
             mbar_init(&bars->q_full[s], 1);
             mbar_init(&bars->q_empty[s], 1);
             mbar_init(&bars->s_full[s], 1);
@@ -161,6 +106,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&bars->o_done[s], 1);
         }
         mbar_init(&bars->drain, 1);
+        mbar_init(&bars->tmem_free, 256);
         bars->abort_flag = 0;
         fence_barrier_init();
         tma_prefetch_desc(&tq);
@@ -177,93 +123,124 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = bars->tmem_slot;
 
-    Sched sc;
-    sc.total = total_tiles;
-    sc.stride = 2 * gridDim.x;
-    sc.base = 2 * blockIdx.x;
-    sc.round[0] = sc.round[1] = 0;
-
+    if (warp < 4) regs_dec<kRegsLow>();
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
-        if (lane == 0) {
-            uint32_t ring = 0, qcount[2] = {0, 0};
-            bool ok = true;
-            unsigned bad = 0;
-            auto load_q = [&](int s) {
-                Tile T = decode_tile(a, sc.tile[s]);
-                ok = ok && mbar_wait(&bars->q_empty[s], (qcount[s] & 1) ^ 1, abort_flag, a.err);
-                if (!ok) return;
-                ++qcount[s];
-                uint8_t* dst = smem + C::OFF_Q + s * C::Q_BYTES;
-                mbar_arrive_expect_tx(&bars->q_full[s], C::Q_BYTES);
-                const int tok0 = PAGED ? a.cu_seqlens[T.b] : 0;
+        // The whole warp walks the schedule (uniform control flow); lane 0 tests barriers and
+        // issues the copies, and all lanes stage list entries into shared memory in bulk.
+        TileIter rit[2], qit[2];     // K/V ring walk and Q walk of each slot
+        int ld[2] = {0, 0};          // next load of the ring tile: K0 V0 K1 V1 ...
+        int lbase[2] = {-1, -1};     // first list entry staged in bars->lst[s]
+        uint32_t ring[2] = {0, 0}, qc[2] = {0, 0};
+        unsigned bad = 0;
+        bool ok = true;
+        for (int s = 0; s < 2; ++s) {
+            rit[s].init(s, base, stride, total_tiles);
+            rit[s].next(a);
+            qit[s] = rit[s];
+        }
+        int idle = 0;
+        long long t_idle = 0;
+        while (ok && (rit[0].active || rit[1].active || qit[0].active || qit[1].active)) {
+            bool prog = false;
 #pragma unroll
-                for (int p = 0; p < C::QP; ++p)
-                    tma_load_4d(dst + p * kBM * 128, &tq, &bars->q_full[s], p * C::PW, tok0 + T.i * a.block, T.h,
-                                PAGED ? 0 : T.b);
-            };
-            auto load_kv = [&](int s, int k, bool is_v) {
-                Tile T = decode_tile(a, sc.tile[s]);
-                int j = list_entry(a, T, k);
-                if (j < 0) {
-                    bad = 1;
-                    j = 0;
-                }
-                const int st = ring % C::NS;
-                ok = ok && mbar_wait(&bars->kv_empty[st], ((ring / C::NS) & 1) ^ 1, abort_flag, a.err);
-                if (!ok) return;
-                ++ring;
-                uint8_t* dst = smem + C::OFF_RING + st * C::KV_BYTES;
-                const CUtensorMap* map = is_v ? &tv : &tk;
-                mbar_arrive_expect_tx(&bars->kv_full[st], C::KV_BYTES);
-#pragma unroll
-                for (int p = 0; p < C::QP; ++p) {
-                    if constexpr (PAGED) {
-#pragma unroll
-                        for (int pg = 0; pg < BN / 64; ++pg) {
-                            const int lp = j * (BN / 64) + pg;
-                            const int phys = lp * 64 < T.n_tok
-                                                 ? __ldg(a.page_table + static_cast<int64_t>(T.b) * a.max_pages + lp)
-                                                 : a.num_pages;  // past the end of the sequence: zeros
-                            tma_load_4d(dst + p * BN * 128 + pg * 64 * 128, map, &bars->kv_full[st], p * C::PW, 0,
-                                        T.hk, phys);
-                        }
-                    } else {
-                        tma_load_4d(dst + p * BN * 128, map, &bars->kv_full[st], p * C::PW, j * a.block, T.hk, T.b);
-                    }
-                }
-            };
             for (int s = 0; s < 2; ++s) {
-                sc.start(a, s);
-                if (sc.active[s]) {
-                    load_q(s);
-                    load_kv(s, 0, false);
-                    sc.a[s] = 1;
+                if (qit[s].active) {
+                    const bool qready = __shfl_sync(0xFFFFFFFFu, lane == 0 ? mbar_test(&bars->q_empty[s], (qc[s] & 1) ^ 1) : 0u, 0);
+                    if (qready) {
+                        if (lane == 0) {
+                            const Tile& T = qit[s].T;
+                            uint8_t* dst = smem + C::OFF_Q + s * C::Q_BYTES;
+                            mbar_arrive_expect_tx(&bars->q_full[s], C::Q_BYTES);
+                            const int tok0 = PAGED ? a.cu_seqlens[T.b] : 0;
+#pragma unroll
+                            for (int p = 0; p < C::QP; ++p)
+                                tma_load_4d(dst + p * kBM * 128, &tq, &bars->q_full[s], p * C::PW, tok0 + T.i * a.block,
+                                            T.h, PAGED ? 0 : T.b);
+                        }
+                        ++qc[s];
+                        qit[s].next(a);
+                        prog = true;
+                    }
                 }
-            }
-            while (ok && (sc.active[0] || sc.active[1])) {
-                for (int s = 0; s < 2 && ok; ++s) {
-                    if (!sc.active[s]) continue;
-                    load_kv(s, sc.a[s] - 1, true);  // V for PV(a-1)
-                    if (sc.a[s] < sc.n[s]) {
-                        load_kv(s, sc.a[s], false);  // K for S(a)
-                        sc.a[s]++;
-                    } else {
-                        sc.start(a, s);
-                        if (sc.active[s]) {
-                            load_q(s);
-                            load_kv(s, 0, false);
-                            sc.a[s] = 1;
+                if (!rit[s].active) continue;
+                const Tile& T = rit[s].T;
+                const int kb = ld[s] >> 1;
+                if (lbase[s] < 0 || kb >= lbase[s] + kListChunk) {
+                    // Stage entries kb .. kb+127 of this tile's list.
+                    __syncwarp();
+                    for (int e = lane; e < kListChunk; e += 32)
+                        if (kb + e < T.n_list) bars->lst[s][e] = list_entry(a, T, kb + e);
+                    lbase[s] = kb;
+                    __syncwarp();
+                }
+                const int st = ring[s] % C::NSS;
+                const bool sready =
+                    __shfl_sync(0xFFFFFFFFu, lane == 0 ? mbar_test(&bars->kv_empty[s][st], ((ring[s] / C::NSS) & 1) ^ 1) : 0u, 0);
+                if (!sready) continue;
+                if (lane == 0) {
+                    const bool is_v = ld[s] & 1;
+                    int j = bars->lst[s][kb - lbase[s]];
+                    if (j < 0) {
+                        bad = 1;
+                        j = 0;
+                    }
+                    uint8_t* dst = smem + C::OFF_RING + (s * C::NSS + st) * C::KV_BYTES;
+                    const CUtensorMap* map = is_v ? &tv : &tk;
+                    uint64_t* fb = &bars->kv_full[s][st];
+                    mbar_arrive_expect_tx(fb, C::KV_BYTES);
+#pragma unroll
+                    for (int p = 0; p < C::QP; ++p) {
+                        if constexpr (PAGED) {
+#pragma unroll
+                            for (int pg = 0; pg < BN / 64; ++pg) {
+                                const int lp = j * (BN / 64) + pg;
+                                const int phys =
+                                    lp * 64 < T.n_tok ? __ldg(a.page_table + static_cast<int64_t>(T.b) * a.max_pages + lp)
+                                                      : a.num_pages;  // past the end of the sequence: zeros
+                                tma_load_4d(dst + p * BN * 128 + pg * 64 * 128, map, fb, p * C::PW, 0, T.hk, phys);
+                            }
+                        } else {
+                            tma_load_4d(dst + p * BN * 128, map, fb, p * C::PW, j * a.block, T.hk, T.b);
                         }
                     }
                 }
+                ++ring[s];
+                if (++ld[s] == 2 * T.n_list) {
+                    ld[s] = 0;
+                    lbase[s] = -1;
+                    rit[s].next(a);
+                }
+                prog = true;
             }
+            if (prog) {
+                idle = 0;
+            } else {
+                if (++idle == 1) t_idle = clock64();
+                if ((idle & 255) == 0) {
+                    if (*abort_flag) {
+                        ok = false;
+                    } else if (clock64() - t_idle > kPollLimitCycles) {
+                        if (lane == 0) {
+                            *abort_flag = 1;
+                            atomicOr(a.err, kDevErrTimeout);
+                        }
+                        ok = false;
+                    }
+                    ok = __all_sync(0xFFFFFFFFu, ok);
+                }
+                __nanosleep(20);
+            }
+        }
+        if (lane == 0) {
             if (bad) atomicOr(a.err, kDevErrInvalidList);
             // Every issued copy must land before the CTA's shared memory goes away.
             volatile int no_abort = 0;
-            const uint32_t issued = ring;
-            for (uint32_t r = issued > C::NS ? issued - C::NS : 0; r < issued; ++r)
-                mbar_wait(&bars->kv_full[r % C::NS], (r / C::NS) & 1, &no_abort, a.err);
+            for (int s = 0; s < 2; ++s) {
+                for (uint32_t r = ring[s] > C::NSS ? ring[s] - C::NSS : 0; r < ring[s]; ++r)
+                    mbar_wait(&bars->kv_full[s][r % C::NSS], (r / C::NSS) & 1, &no_abort, a.err);
+                if (qc[s] > 0) mbar_wait(&bars->q_full[s], (qc[s] - 1) & 1, &no_abort, a.err);
+            }
         }
         __syncwarp();
     } else if (warp == 1) {
@@ -271,104 +248,135 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             const uint32_t idesc_s = make_idesc(kBM, BN, FP8 ? 0u : 1u, false, false);
             const uint32_t idesc_o = make_idesc(kBM, D, FP8 ? 0u : 1u, false, true);
-            uint32_t ring = 0, qcount[2] = {0, 0}, pcount[2] = {0, 0};
+            TileIter it[2];
+            int kblk[2] = {0, 0};
+            bool need_s[2] = {true, true}, q_seen[2] = {false, false}, p_seen[2] = {false, false};
+            uint32_t rc[2] = {0, 0}, qc[2] = {0, 0}, pc[2] = {0, 0}, pv_issued[2] = {0, 0}, oc[2] = {0, 0};
             bool ok = true;
-            auto mma_s = [&](int s) {
-                if (sc.a[s] == 0) {  // first block of a tile: its Q must have landed
-                    ok = ok && mbar_wait(&bars->q_full[s], qcount[s] & 1, abort_flag, a.err);
-                    ++qcount[s];
-                }
-                const int st = ring % C::NS;
-                ok = ok && mbar_wait(&bars->kv_full[st], (ring / C::NS) & 1, abort_flag, a.err);
-                if (!ok) return;
-                ++ring;
-                tc_fence_after();
-                const uint32_t aQ = smem_u32(smem + C::OFF_Q + s * C::Q_BYTES);
-                const uint32_t aK = smem_u32(smem + C::OFF_RING + st * C::KV_BYTES);
-#pragma unroll
-                for (int kk = 0; kk < C::KSTEPS_S; ++kk) {
-                    const uint32_t byte = kk * 32, pan = byte / 128, within = byte % 128;
-                    const uint64_t da = smem_desc_sw128(aQ + pan * kBM * 128 + within, 16, 1024);
-                    const uint64_t db = smem_desc_sw128(aK + pan * BN * 128 + within, 16, 1024);
-                    if constexpr (FP8)
-                        mma_f8_ss(tmem + s * 128, da, db, idesc_s, kk > 0);
-                    else
-                        mma_f16_ss(tmem + s * 128, da, db, idesc_s, kk > 0);
-                }
-                tc_commit(&bars->kv_empty[st]);
-                tc_commit(&bars->s_full[s]);
-                if (sc.a[s] == sc.n[s] - 1) tc_commit(&bars->q_empty[s]);  // last S of the tile
-            };
-            auto mma_pv = [&](int s, int k) {
-                ok = ok && mbar_wait(&bars->p_full[s], pcount[s] & 1, abort_flag, a.err);
-                ++pcount[s];
-                const int st = ring % C::NS;
-                ok = ok && mbar_wait(&bars->kv_full[st], (ring / C::NS) & 1, abort_flag, a.err);
-                if (!ok) return;
-                ++ring;
-                tc_fence_after();
-                const uint32_t aP = smem_u32(smem + C::OFF_P + s * C::P_BYTES);
-                const uint32_t aV = smem_u32(smem + C::OFF_RING + st * C::KV_BYTES);
-#pragma unroll
-                for (int kk = 0; kk < C::KSTEPS_O; ++kk) {
-                    const uint32_t byte = kk * 32, pan = byte / 128, within = byte % 128;
-                    const uint64_t da = smem_desc_sw128(aP + pan * kBM * 128 + within, 16, 1024);
-                    const uint64_t db = smem_desc_sw128(aV + kk * C::ROWS_PER_KSTEP * 128, BN * 128, 1024);
-                    const uint32_t acc = (k > 0 || kk > 0) ? 1u : 0u;
-                    if constexpr (FP8)
-                        mma_f8_ss(tmem + 256 + s * 128, da, db, idesc_o, acc);
-                    else
-                        mma_f16_ss(tmem + 256 + s * 128, da, db, idesc_o, acc);
-                }
-                tc_commit(&bars->kv_empty[st]);
-                tc_commit(&bars->o_done[s]);
-            };
             for (int s = 0; s < 2; ++s) {
-                sc.start(a, s);
-                if (sc.active[s]) {
-                    mma_s(s);
-                    sc.a[s] = 1;
-                }
+                it[s].init(s, base, stride, total_tiles);
+                it[s].next(a);
             }
-            while (ok && (sc.active[0] || sc.active[1])) {
-                for (int s = 0; s < 2 && ok; ++s) {
-                    if (!sc.active[s]) continue;
-                    mma_pv(s, sc.a[s] - 1);
-                    if (sc.a[s] < sc.n[s]) {
-                        mma_s(s);
-                        sc.a[s]++;
+            int idle = 0;
+            long long t_idle = 0;
+            while (ok && (it[0].active || it[1].active)) {
+                bool prog = false;
+#pragma unroll
+                for (int s = 0; s < 2; ++s) {
+                    if (!it[s].active) continue;
+                    const int st = rc[s] % C::NSS;
+                    if (need_s[s]) {
+                        // S(k) = Q K^T: its Q has landed, its K stage is full, and the previous
+                        // PV (which reads P from these TMEM columns) is complete.
+                        if (kblk[s] == 0 && !q_seen[s]) {
+                            if (!mbar_test(&bars->q_full[s], qc[s] & 1)) continue;
+                            q_seen[s] = true;
+                            ++qc[s];
+                        }
+                        if (oc[s] < pv_issued[s]) {
+                            if (!mbar_test(&bars->o_done[s], oc[s] & 1)) continue;
+                            ++oc[s];
+                        }
+                        if (!mbar_test(&bars->kv_full[s][st], (rc[s] / C::NSS) & 1)) continue;
+                        tc_fence_after();
+                        const uint32_t aQ = smem_u32(smem + C::OFF_Q + s * C::Q_BYTES);
+                        const uint32_t aK = smem_u32(smem + C::OFF_RING + (s * C::NSS + st) * C::KV_BYTES);
+#pragma unroll
+                        for (int kk = 0; kk < C::KSTEPS_S; ++kk) {
+                            const uint32_t byte = kk * 32, pan = byte / 128, within = byte % 128;
+                            const uint64_t da = smem_desc_sw128(aQ + pan * kBM * 128 + within, 16, 1024);
+                            const uint64_t db = smem_desc_sw128(aK + pan * BN * 128 + within, 16, 1024);
+                            if constexpr (FP8)
+                                mma_f8_ss(tmem + s * 128, da, db, idesc_s, kk > 0);
+                            else
+                                mma_f16_ss(tmem + s * 128, da, db, idesc_s, kk > 0);
+                        }
+                        tc_commit(&bars->kv_empty[s][st]);
+                        tc_commit(&bars->s_full[s]);
+                        if (kblk[s] == it[s].T.n_list - 1) {
+                            tc_commit(&bars->q_empty[s]);  // last S of the tile: Q_s may be reloaded
+                            q_seen[s] = false;
+                        }
+                        ++rc[s];
+                        need_s[s] = false;
+                        prog = true;
                     } else {
-                        sc.start(a, s);
-                        if (sc.active[s]) {
-                            mma_s(s);
-                            sc.a[s] = 1;
+                        // O += P V: P written to TMEM by the softmax, V stage full.
+                        if (!p_seen[s]) {
+                            if (!mbar_test(&bars->p_full[s], pc[s] & 1)) continue;
+                            p_seen[s] = true;
+                            ++pc[s];
+                        }
+                        if (!mbar_test(&bars->kv_full[s][st], (rc[s] / C::NSS) & 1)) continue;
+                        tc_fence_after();
+                        const uint32_t aV = smem_u32(smem + C::OFF_RING + (s * C::NSS + st) * C::KV_BYTES);
+#pragma unroll
+                        for (int kk = 0; kk < C::KSTEPS_O; ++kk) {
+                            const uint64_t db = smem_desc_sw128(aV + kk * C::ROWS_PER_KSTEP * 128, BN * 128, 1024);
+                            const uint32_t acc = (kblk[s] > 0 || kk > 0) ? 1u : 0u;
+                            if constexpr (FP8)
+                                mma_f8_ts(tmem + 256 + s * 128, tmem + s * 128 + kk * 8, db, idesc_o, acc);
+                            else
+                                mma_f16_ts(tmem + 256 + s * 128, tmem + s * 128 + kk * 8, db, idesc_o, acc);
+                        }
+                        tc_commit(&bars->kv_empty[s][st]);
+                        tc_commit(&bars->o_done[s]);
+                        ++pv_issued[s];
+                        ++rc[s];
+                        p_seen[s] = false;
+                        need_s[s] = true;
+                        if (++kblk[s] == it[s].T.n_list) {
+                            kblk[s] = 0;
+                            it[s].next(a);
+                        }
+                        prog = true;
+                    }
+                }
+                if (prog) {
+                    idle = 0;
+                } else {
+                    if (++idle == 1) t_idle = clock64();
+                    if ((idle & 255) == 0) {
+                        if (*abort_flag) {
+                            ok = false;
+                        } else if (clock64() - t_idle > kPollLimitCycles) {
+                            *abort_flag = 1;
+                            atomicOr(a.err, kDevErrTimeout);
+                            ok = false;
                         }
                     }
+                    __nanosleep(20);
                 }
             }
             // Drain: wait until every MMA issued by this thread has completed.
             tc_commit(&bars->drain);
             volatile int no_abort = 0;
             mbar_wait(&bars->drain, 0, &no_abort, a.err);
+            // Every softmax thread has finished with TMEM (bounded: the softmax warps exit
+            // their loops on abort too).
+            mbar_wait(&bars->tmem_free, 0, &no_abort, a.err);
         }
         __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+        return;
     } else if (warp >= 4) {
         // ------------------------------------------------------------ softmax, slot s
+        regs_inc<kRegsHigh>();
         const int s = (warp - 4) / 4;
         const int quad = warp % 4;
         const int row = quad * 32 + lane;
         const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-        const uint32_t tS = tmem + lane_base + s * 128;
+        const uint32_t tS = tmem + lane_base + s * 128;  // S, then P in place
         const uint32_t tO = tmem + lane_base + 256 + s * 128;
-        uint8_t* sP = smem + C::OFF_P + s * C::P_BYTES;
         uint32_t scount = 0, ocount = 0;
         const float sl2 = a.scale_log2;
         bool ok = true;
-        for (int r = 0; ok; ++r) {
-            const int t = sc.base + s + r * sc.stride;
-            if (t >= total_tiles) break;
-            Tile T = decode_tile(a, t);
-            if (!T.valid || T.n_list == 0) continue;
+        TileIter it;
+        it.init(s, base, stride, total_tiles);
+        it.next(a);
+        while (ok && it.active) {
+            const Tile T = it.T;
             float m_used = -INFINITY, l_run = 0.f;
             int j_next = list_entry(a, T, 0);
             for (int k = 0; k < T.n_list; ++k) {
@@ -384,39 +392,37 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 // Only the diagonal block needs the causal mask (and an out-of-range entry, all -inf).
                 const bool diag = (j == T.i);
-                // Pass 1: row max, 64 TMEM columns per load, eight independent max chains.
+                // The whole S row in registers: one TMEM round trip per block.
+                uint32_t rr[BN];
+                if constexpr (BN == 128)
+                    tmem_ld128(tS, rr);
+                else
+                    tmem_ld64(tS, rr);
+                // Row max with eight independent chains.
                 float mx = -INFINITY;
                 if (j >= 0) {
                     float m8[8];
 #pragma unroll
                     for (int q = 0; q < 8; ++q) m8[q] = -INFINITY;
+                    if (!diag) {
 #pragma unroll
-                    for (int hf = 0; hf < BN / 64; ++hf) {
-                        uint32_t rr[64];
-                        tmem_ld64(tS + hf * 64, rr);
-                        if (!diag) {
+                        for (int e = 0; e < BN; e += 2)
+                            m8[(e / 2) % 8] = max3f(m8[(e / 2) % 8], __uint_as_float(rr[e]), __uint_as_float(rr[e + 1]));
+                    } else {
 #pragma unroll
-                            for (int e = 0; e < 64; e += 2)
-                                m8[(e / 2) % 8] = max3f(m8[(e / 2) % 8], __uint_as_float(rr[e]), __uint_as_float(rr[e + 1]));
-                        } else {
-#pragma unroll
-                            for (int e = 0; e < 64; ++e)
-                                if (hf * 64 + e <= row) m8[e % 8] = fmaxf(m8[e % 8], __uint_as_float(rr[e]));
-                        }
+                        for (int e = 0; e < BN; ++e)
+                            if (e <= row) m8[e % 8] = fmaxf(m8[e % 8], __uint_as_float(rr[e]));
                     }
                     mx = max3f(max3f(m8[0], m8[1], m8[2]), max3f(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
                 }
                 const float m_blk = mx * sl2;
-                // The running max is refreshed only when a block's max exceeds it by more than
-                // kRescaleLog2 (log2 units); P is formed as 2^(s - m) * kPScale, so P <= 2^(8) stays
-                // inside BF16 and E4M3, and the O rescale below is rare.
                 float m_new = m_used;
                 if (m_blk > m_used + kRescaleLog2<FP8>) m_new = m_blk;
                 const float alpha = (m_new == m_used) ? 1.f : fast_exp2(m_used - m_new);
-                // exp2(s * sl2 - mref) = 2^(s - m_new) * kPScale
+                // exp2(s * sl2 - mref) = 2^(s - m_new) * P scale
                 const float mref = (m_new == -INFINITY) ? 0.f : m_new - kPScaleLog2<FP8>;
                 if (k > 0) {
-                    // PV(k-1) must be done: it reads P_s (rewritten below) and writes O_s.
+                    // PV(k-1) writes O_s: it must be done before the rescale below.
                     w_ok = mbar_wait(&bars->o_done[s], ocount & 1, abort_flag, a.err);
                     ++ocount;
                     w_ok = __all_sync(0xFFFFFFFFu, w_ok);
@@ -428,65 +434,68 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (__any_sync(0xFFFFFFFFu, alpha != 1.f)) {
 #pragma unroll 1
                         for (int ch = 0; ch < D / 32; ++ch) {
-                            uint32_t rr[32];
-                            tmem_ld32(tO + ch * 32, rr);
+                            uint32_t ro[32];
+                            tmem_ld32(tO + ch * 32, ro);
 #pragma unroll
-                            for (int e = 0; e < 32; ++e) rr[e] = __float_as_uint(__uint_as_float(rr[e]) * alpha);
-                            tmem_st32(tO + ch * 32, rr);
+                            for (int e = 0; e < 32; ++e) ro[e] = __float_as_uint(__uint_as_float(ro[e]) * alpha);
+                            tmem_st32(tO + ch * 32, ro);
                         }
-                        tmem_st_wait();
                     }
                 }
-                // Pass 2: P = exp2(S * sl2 - mref) on packed pairs, four packed partial sums, and
-                // P -> shared memory (128-byte swizzled K-major A operand of the PV MMA).
+                // P = exp2(S * sl2 - mref) on packed pairs, four packed partial sums; P is packed
+                // (BF16 pairs or E4M3 quads) into the first columns of S_s as the TMEM A operand
+                // of the PV MMA (S is already in registers).
                 const uint64_t sl2x2 = pack_f32x2(sl2, sl2);
                 const uint64_t negm = pack_f32x2(-mref, -mref);
+                // Most exponentials on the FMA pipe (polynomial), one pair in eight on MUFU; P is
+                // then packed with one hardware conversion per pair (E4M3 or BF16).
+                constexpr int kDeg = FP8 ? 2 : 3;
                 uint64_t sum4[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-                for (int hf = 0; hf < BN / 64; ++hf) {
-                    uint32_t rr[64];
-                    tmem_ld64(tS + hf * 64, rr);
-                    float pv[64];
-#pragma unroll
-                    for (int e = 0; e < 64; e += 2) {
-                        const uint64_t x = fma_f32x2(pack_f32x2(__uint_as_float(rr[e]), __uint_as_float(rr[e + 1])),
-                                                     sl2x2, negm);
-                        float x0, x1;
-                        unpack_f32x2(x, x0, x1);
-                        pv[e] = fast_exp2(x0);
-                        pv[e + 1] = fast_exp2(x1);
-                    }
+                for (int e = 0; e < BN; e += 2) {
+                    const uint64_t x = fma_f32x2(pack_f32x2(__uint_as_float(rr[e]), __uint_as_float(rr[e + 1])),
+                                                 sl2x2, negm);
+                    float x0, x1;
+                    unpack_f32x2(x, x0, x1);
                     if (diag || j < 0) {
-#pragma unroll
-                        for (int e = 0; e < 64; ++e)
-                            if (j < 0 || hf * 64 + e > row) pv[e] = 0.f;
+                        if (j < 0 || e > row) x0 = -INFINITY;
+                        if (j < 0 || e + 1 > row) x1 = -INFINITY;
                     }
-#pragma unroll
-                    for (int e = 0; e < 64; e += 2)
-                        sum4[(e / 2) % 4] = add_f32x2(sum4[(e / 2) % 4], pack_f32x2(pv[e], pv[e + 1]));
-                    if constexpr (FP8) {
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {  // four 16-key units of e4m3
-                            uint32_t w4[4];
-#pragma unroll
-                            for (int q = 0; q < 4; ++q) {
-                                const int e = u * 16 + q * 4;
-                                w4[q] = pack_e4m3x2(pv[e], pv[e + 1]) | (static_cast<uint32_t>(pack_e4m3x2(pv[e + 2], pv[e + 3])) << 16);
-                            }
-                            const int unit = hf * 4 + u, pan = unit / 8, cc = unit % 8;
-                            *reinterpret_cast<uint4*>(sP + pan * kBM * 128 + row * 128 + ((cc ^ (row & 7)) * 16)) =
-                                make_uint4(w4[0], w4[1], w4[2], w4[3]);
-                        }
+                    float p0, p1;
+                    if ((e / 2) % 8 == 7) {
+                        p0 = fast_exp2(x0);
+                        p1 = fast_exp2(x1);
                     } else {
-#pragma unroll
-                        for (int u = 0; u < 8; ++u) {  // eight 8-key units of bf16
-                            uint32_t w4[4];
-#pragma unroll
-                            for (int q = 0; q < 4; ++q) w4[q] = pack_bf16x2(pv[u * 8 + 2 * q], pv[u * 8 + 2 * q + 1]);
-                            const int unit = hf * 8 + u, pan = unit / 8, cc = unit % 8;
-                            *reinterpret_cast<uint4*>(sP + pan * kBM * 128 + row * 128 + ((cc ^ (row & 7)) * 16)) =
-                                make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                        exp2_poly_x2<kDeg>(x0, x1, p0, p1);
+                        if (diag || j < 0) {  // the polynomial maps -inf to ~2^-126, not 0
+                            if (j < 0 || e > row) p0 = 0.f;
+                            if (j < 0 || e + 1 > row) p1 = 0.f;
                         }
+                    }
+                    sum4[(e / 2) % 4] = add_f32x2(sum4[(e / 2) % 4], pack_f32x2(p0, p1));
+                    rr[e] = __float_as_uint(p0);
+                    rr[e + 1] = __float_as_uint(p1);
+                }
+                if constexpr (FP8) {
+                    uint32_t pk[BN / 4];
+#pragma unroll
+                    for (int q = 0; q < BN / 4; ++q)
+                        pk[q] = pack_e4m3x2(__uint_as_float(rr[4 * q]), __uint_as_float(rr[4 * q + 1])) |
+                                (static_cast<uint32_t>(pack_e4m3x2(__uint_as_float(rr[4 * q + 2]),
+                                                                   __uint_as_float(rr[4 * q + 3])))
+                                 << 16);
+                    if constexpr (BN == 128)
+                        tmem_st32(tS, pk);
+                    else
+                        tmem_st16(tS, pk);
+                } else {
+#pragma unroll
+                    for (int hf = 0; hf < BN / 64; ++hf) {
+                        uint32_t pk[32];
+#pragma unroll
+                        for (int q = 0; q < 32; ++q)
+                            pk[q] = pack_bf16x2(__uint_as_float(rr[hf * 64 + 2 * q]), __uint_as_float(rr[hf * 64 + 2 * q + 1]));
+                        tmem_st32(tS + hf * 32, pk);
                     }
                 }
                 float s0, s1, s2, s3, s4, s5, s6, s7;
@@ -497,7 +506,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float sum = ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
                 l_run = l_run * alpha + sum;
                 m_used = m_new;
-                fence_proxy_async_smem();
+                tmem_st_wait();
                 tc_fence_before();
                 mbar_arrive(&bars->p_full[s]);
             }
@@ -534,15 +543,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (store && a.lse != nullptr)
                 a.lse[(static_cast<int64_t>(T.b) * a.Hq + T.h) * a.lse_stride + t_row] =
                     (m_used + __log2f(l_run) - kPScaleLog2<FP8>) * 0.69314718055994531f;
-            // The next tile's first PV overwrites O_s; its p_full arrival (after these loads)
-            // is what lets the MMA warp issue it.
+            // The next tile's first PV overwrites O_s; the p_full arrival that lets the MMA warp
+            // issue it comes after these loads.
             tc_fence_before();
+            it.next(a);
         }
+        tc_fence_before();
+        mbar_arrive(&bars->tmem_free);
+        return;
     }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
 template <bool FP8, int D, int BN, bool PAGED>

@@ -62,6 +62,15 @@ struct AttnArgs {
     unsigned* err;
 };
 
+// Persistent, two independent pipelined CTAs per SM, one query tile each (attn_ws2.cu).
+cudaError_t launch_attention_ws2(bool fp8, bool paged, const CUtensorMap& tq, const CUtensorMap& tk,
+                                 const CUtensorMap& tv, const AttnArgs& a, cudaStream_t s);
+
+// As ws2, but P goes through shared memory so S(k+1) is computed while the softmax still works
+// on block k (attn_ws3.cu).  FP8, and BF16 shapes whose stages fit two CTAs per SM.
+cudaError_t launch_attention_ws3(bool fp8, bool paged, const CUtensorMap& tq, const CUtensorMap& tk,
+                                 const CUtensorMap& tv, const AttnArgs& a, cudaStream_t s);
+
 // Sets the message bsa_last_error() returns on this thread.
 void set_last_error(const char* msg);
 
