@@ -55,11 +55,12 @@ struct Cfg3 {
 };
 
 // BF16: refresh the running max only when it grows by more than 2^8 (P <= 256 unscaled);
-// E4M3: beyond 2^3 with P scaled by 2^5, so P <= 2^8 fits E4M3 with room below.
+// E4M3: beyond 2^5 with P scaled by 2^3, so P <= 2^8 fits E4M3 and values down to 2^-12 of the
+// row max keep E4M3 precision.
 template <bool FP8>
-constexpr float kRescale3 = FP8 ? 3.f : 8.f;
+constexpr float kRescale3 = FP8 ? 5.f : 8.f;
 template <bool FP8>
-constexpr float kPScale3 = FP8 ? 5.f : 0.f;
+constexpr float kPScale3 = FP8 ? 3.f : 0.f;
 
 struct Bars3 {
     uint64_t kv_full[kMaxStages3], kv_empty[kMaxStages3];
@@ -304,25 +305,27 @@ __global__ void __launch_bounds__(kThreads3, 2)
                 }
                 tc_fence_after();
                 const bool diag = (j == T.i);
-                // Pass 1: row max, 64 TMEM columns per load, eight independent max chains.
+                // The whole S row in registers with one TMEM read; after it S may be overwritten.
+                uint32_t rr[BN];
+                if constexpr (BN == 128)
+                    tmem_ld128(tS, rr);
+                else
+                    tmem_ld64(tS, rr);
+                tc_fence_before();
+                mbar_arrive(&bars->s_free);
                 float mx = -INFINITY;
                 if (j >= 0) {
                     float m8[8];
 #pragma unroll
                     for (int q = 0; q < 8; ++q) m8[q] = -INFINITY;
+                    if (!diag) {
 #pragma unroll
-                    for (int hf = 0; hf < BN / 64; ++hf) {
-                        uint32_t rr[64];
-                        tmem_ld64(tS + hf * 64, rr);
-                        if (!diag) {
+                        for (int e = 0; e < BN; e += 2)
+                            m8[(e / 2) % 8] = max3f(m8[(e / 2) % 8], __uint_as_float(rr[e]), __uint_as_float(rr[e + 1]));
+                    } else {
 #pragma unroll
-                            for (int e = 0; e < 64; e += 2)
-                                m8[(e / 2) % 8] = max3f(m8[(e / 2) % 8], __uint_as_float(rr[e]), __uint_as_float(rr[e + 1]));
-                        } else {
-#pragma unroll
-                            for (int e = 0; e < 64; ++e)
-                                if (hf * 64 + e <= row) m8[e % 8] = fmaxf(m8[e % 8], __uint_as_float(rr[e]));
-                        }
+                        for (int e = 0; e < BN; ++e)
+                            if (e <= row) m8[e % 8] = fmaxf(m8[e % 8], __uint_as_float(rr[e]));
                     }
                     mx = max3f(max3f(m8[0], m8[1], m8[2]), max3f(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
                 }
@@ -331,6 +334,25 @@ __global__ void __launch_bounds__(kThreads3, 2)
                 if (m_blk > m_used + kRescale3<FP8>) m_new = m_blk;
                 const float alpha = (m_new == m_used) ? 1.f : fast_exp2(m_used - m_new);
                 const float mref = (m_new == -INFINITY) ? 0.f : m_new - kPScale3<FP8>;
+                // P = exp2(S * sl2 - mref) in place, four packed partial sums.
+                const uint64_t sl2x2 = pack_f32x2(sl2, sl2);
+                const uint64_t negm = pack_f32x2(-mref, -mref);
+                uint64_t sum4[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+                for (int e = 0; e < BN; e += 2) {
+                    const uint64_t x = fma_f32x2(pack_f32x2(__uint_as_float(rr[e]), __uint_as_float(rr[e + 1])),
+                                                 sl2x2, negm);
+                    float x0, x1;
+                    unpack_f32x2(x, x0, x1);
+                    float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+                    if (diag || j < 0) {
+                        if (j < 0 || e > row) p0 = 0.f;
+                        if (j < 0 || e + 1 > row) p1 = 0.f;
+                    }
+                    sum4[(e / 2) % 4] = add_f32x2(sum4[(e / 2) % 4], pack_f32x2(p0, p1));
+                    rr[e] = __float_as_uint(p0);
+                    rr[e + 1] = __float_as_uint(p1);
+                }
                 if (k > 0) {
                     // PV(k-1) reads P (rewritten below) and writes O (maybe rescaled below).
                     w_ok = mbar_wait(&bars->o_done, ocount & 1, abort_flag, a.err);
@@ -342,61 +364,32 @@ __global__ void __launch_bounds__(kThreads3, 2)
                     }
                     tc_fence_after();
                 }
-                // Pass 2: P = exp2(S * sl2 - mref), 64 columns at a time, written to shared memory
-                // in the 128-byte-swizzled K-major layout of the PV A operand.  Once the last S
-                // columns are in registers the MMA warp may overwrite S with the next block's.
-                const uint64_t sl2x2 = pack_f32x2(sl2, sl2);
-                const uint64_t negm = pack_f32x2(-mref, -mref);
-                uint64_t sum4[4] = {0ull, 0ull, 0ull, 0ull};
+                // P -> shared memory in the 128-byte-swizzled K-major layout of the PV A operand.
+                if constexpr (FP8) {
 #pragma unroll
-                for (int hf = 0; hf < BN / 64; ++hf) {
-                    uint32_t rr[64];
-                    tmem_ld64(tS + hf * 64, rr);
-                    if (hf == BN / 64 - 1) {
-                        tc_fence_before();
-                        mbar_arrive(&bars->s_free);
+                    for (int unit = 0; unit < BN / 16; ++unit) {  // 16 keys of e4m3 per 16 bytes
+                        uint32_t w4[4];
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const int e = unit * 16 + q * 4;
+                            w4[q] = pack_e4m3x2(__uint_as_float(rr[e]), __uint_as_float(rr[e + 1])) |
+                                    (static_cast<uint32_t>(pack_e4m3x2(__uint_as_float(rr[e + 2]), __uint_as_float(rr[e + 3])))
+                                     << 16);
+                        }
+                        const int pan = unit / 8, cc = unit % 8;
+                        *reinterpret_cast<uint4*>(sP + pan * kBM3 * 128 + row * 128 + ((cc ^ (row & 7)) * 16)) =
+                            make_uint4(w4[0], w4[1], w4[2], w4[3]);
                     }
+                } else {
 #pragma unroll
-                    for (int e = 0; e < 64; e += 2) {
-                        const uint64_t x = fma_f32x2(pack_f32x2(__uint_as_float(rr[e]), __uint_as_float(rr[e + 1])),
-                                                     sl2x2, negm);
-                        float x0, x1;
-                        unpack_f32x2(x, x0, x1);
-                        float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
-                        if (diag || j < 0) {
-                            if (j < 0 || hf * 64 + e > row) p0 = 0.f;
-                            if (j < 0 || hf * 64 + e + 1 > row) p1 = 0.f;
-                        }
-                        sum4[(e / 2) % 4] = add_f32x2(sum4[(e / 2) % 4], pack_f32x2(p0, p1));
-                        rr[e] = __float_as_uint(p0);
-                        rr[e + 1] = __float_as_uint(p1);
-                    }
-                    if constexpr (FP8) {
+                    for (int unit = 0; unit < BN / 8; ++unit) {  // 8 keys of bf16 per 16 bytes
+                        uint32_t w4[4];
 #pragma unroll
-                        for (int u = 0; u < 4; ++u) {  // four 16-key units of e4m3
-                            uint32_t w4[4];
-#pragma unroll
-                            for (int q = 0; q < 4; ++q) {
-                                const int e = u * 16 + q * 4;
-                                w4[q] = pack_e4m3x2(__uint_as_float(rr[e]), __uint_as_float(rr[e + 1])) |
-                                        (static_cast<uint32_t>(pack_e4m3x2(__uint_as_float(rr[e + 2]), __uint_as_float(rr[e + 3])))
-                                         << 16);
-                            }
-                            const int unit = hf * 4 + u, pan = unit / 8, cc = unit % 8;
-                            *reinterpret_cast<uint4*>(sP + pan * kBM3 * 128 + row * 128 + ((cc ^ (row & 7)) * 16)) =
-                                make_uint4(w4[0], w4[1], w4[2], w4[3]);
-                        }
-                    } else {
-#pragma unroll
-                        for (int u = 0; u < 8; ++u) {  // eight 8-key units of bf16
-                            uint32_t w4[4];
-#pragma unroll
-                            for (int q = 0; q < 4; ++q)
-                                w4[q] = pack_bf16x2(__uint_as_float(rr[u * 8 + 2 * q]), __uint_as_float(rr[u * 8 + 2 * q + 1]));
-                            const int unit = hf * 8 + u, pan = unit / 8, cc = unit % 8;
-                            *reinterpret_cast<uint4*>(sP + pan * kBM3 * 128 + row * 128 + ((cc ^ (row & 7)) * 16)) =
-                                make_uint4(w4[0], w4[1], w4[2], w4[3]);
-                        }
+                        for (int q = 0; q < 4; ++q)
+                            w4[q] = pack_bf16x2(__uint_as_float(rr[unit * 8 + 2 * q]), __uint_as_float(rr[unit * 8 + 2 * q + 1]));
+                        const int pan = unit / 8, cc = unit % 8;
+                        *reinterpret_cast<uint4*>(sP + pan * kBM3 * 128 + row * 128 + ((cc ^ (row & 7)) * 16)) =
+                            make_uint4(w4[0], w4[1], w4[2], w4[3]);
                     }
                 }
                 fence_proxy_async_smem();
