@@ -141,6 +141,23 @@ def whole_job_tflops(eff_flop_per_rank: float, world: int, ms_per_step: float) -
     return eff_flop_per_rank * world / (ms_per_step * 1e-3) / 1e12
 
 
+# DRAM bytes per token moved by one bsa_prefill launch (dram__bytes_read.sum +
+# dram__bytes_write.sum of one ncu capture on the fp8-32k workload, divided by its 32768
+# tokens).  Q, K, V are read and O written once per token, so the traffic of a launch is
+# linear in B x N.  Keyed by attention kernel and (dtype, Hq, Hkv, d) of the capture; any
+# other kernel or shape reports null.
+TRAFFIC_PER_TOKEN = {
+    ("serial", "fp8", 64, 8, 128): (359.159296e6 + 487.020288e6) / 32768,
+}
+ATTN_DEFAULT = "serial"  # the kernel bsa_prefill runs when BSA_ATTN_VARIANT is unset
+
+
+def attn_traffic(fp8: bool, B: int, N: int, Hq: int, Hkv: int, D: int):
+    kern = os.environ.get("BSA_ATTN_VARIANT") or ATTN_DEFAULT
+    per = TRAFFIC_PER_TOKEN.get((kern, "fp8" if fp8 else "bf16", Hq, Hkv, D))
+    return None if per is None else per * B * N
+
+
 def peaks():
     p = ROOT / "MEASURED_PEAKS.json"
     if p.exists():
@@ -428,7 +445,8 @@ def main():
                          "unit": "TFLOP/s", "frac": attn_ach / peak,
                          "peak_source": f"{src} bf16 {'sustained' if 'bf16_tflops_sustained' in pk else 'burst'}"
                                         f"{' x2 (fp8/bf16 nominal ratio)' if fp8 else ''}",
-                         "traffic": None},
+                         "traffic": attn_traffic(fp8, res["B"], res["N"], res["Hq"], res["Hkv"], res["D"]),
+                         "traffic_source": "ncu dram bytes of the fp8-32k capture, scaled by tokens"},
             "gpu_launches": 5 * args.steps,
             "clocks": res["clocks"],
         }
