@@ -3,8 +3,9 @@ causal attention.  The kernels and the C ABI live in libbsa.so (``build.build()`
 it in-tree); this package exposes the ABI's entry points through ``binding``."""
 from .binding import (BSA_BF16, BSA_FP8_E4M3, BSA_FP32, BSA_METRIC_OAM, BSA_METRIC_OAM_MUL, BSA_METRIC_SAM,
                       BsaError, bsa_check_device_error, bsa_prefill, bsa_prefill_paged, bsa_score_workspace_bytes,
-                      bsa_tpd_budget, stem_score, stem_select)
+                      bsa_selftest_wait_timeout, bsa_tpd_budget, stem_score, stem_score_noalloc, stem_select)
 
 __all__ = ["stem_score", "stem_select", "bsa_prefill", "bsa_prefill_paged", "bsa_tpd_budget",
-           "bsa_score_workspace_bytes", "bsa_check_device_error", "BsaError", "BSA_BF16", "BSA_FP8_E4M3",
+           "bsa_score_workspace_bytes", "bsa_check_device_error", "bsa_selftest_wait_timeout", "stem_score_noalloc",
+           "BsaError", "BSA_BF16", "BSA_FP8_E4M3",
            "BSA_FP32", "BSA_METRIC_OAM", "BSA_METRIC_SAM", "BSA_METRIC_OAM_MUL"]

@@ -23,7 +23,8 @@ STATUS = {0: "BSA_OK", 1: "BSA_ERR_INVALID_ARG", 2: "BSA_ERR_UNSUPPORTED", 3: "B
 
 # Every symbol include/bsa.h declares.
 EXPORTS = ["bsa_tpd_budget", "bsa_score_workspace_bytes", "stem_score", "stem_select", "bsa_prefill",
-           "bsa_prefill_paged", "bsa_last_error", "bsa_check_device_error", "stem_score_noalloc"]
+           "bsa_prefill_paged", "bsa_last_error", "bsa_check_device_error", "stem_score_noalloc",
+           "bsa_selftest_wait_timeout"]
 
 
 class BsaError(RuntimeError):
@@ -59,7 +60,9 @@ def lib():
                                     f32, P, P]
     L.bsa_last_error.restype = ctypes.c_char_p
     L.bsa_check_device_error.argtypes = [P]
-    for name in ["stem_score", "stem_score_noalloc", "stem_select", "bsa_prefill", "bsa_prefill_paged", "bsa_check_device_error"]:
+    L.bsa_selftest_wait_timeout.argtypes = [ctypes.c_uint64, P]
+    for name in ["stem_score", "stem_score_noalloc", "stem_select", "bsa_prefill", "bsa_prefill_paged", "bsa_check_device_error",
+                 "bsa_selftest_wait_timeout"]:
         getattr(L, name).restype = ctypes.c_int
     _lib = L
     return L
@@ -204,6 +207,13 @@ def bsa_check_device_error(device=None):
     """Synchronises the current stream and raises if a kernel recorded an error."""
     s = torch.cuda.current_stream(device)
     _check(lib().bsa_check_device_error(ctypes.c_void_p(s.cuda_stream)))
+
+
+def bsa_selftest_wait_timeout(limit_ns: int = 50_000_000, device=None):
+    """Launches the library's wait-timeout self-test kernel on the current stream (see bsa.h);
+    a following bsa_check_device_error() raises BsaError with status BSA_ERR_TIMEOUT."""
+    s = torch.cuda.current_stream(device)
+    _check(lib().bsa_selftest_wait_timeout(int(limit_ns), ctypes.c_void_p(s.cuda_stream)))
 
 
 def nb_of(N: int, block: int) -> int:

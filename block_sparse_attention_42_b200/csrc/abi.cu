@@ -151,6 +151,8 @@ cudaError_t launch_attn(bool fp8, bool paged, const CUtensorMap& tq, const CUten
     if (v && std::strcmp(v, "ws") == 0) return launch_attention_ws(fp8, paged, tq, tk, tv, a, s);
     if (v && std::strcmp(v, "ws2") == 0) return launch_attention_ws2(fp8, paged, tq, tk, tv, a, s);
     if (v && std::strcmp(v, "ws3") == 0) return launch_attention_ws3(fp8, paged, tq, tk, tv, a, s);
+    if (v && std::strcmp(v, "ws4") == 0) return launch_attention_ws4(fp8, paged, tq, tk, tv, a, s);
+    if (v && std::strcmp(v, "pipe") == 0) return launch_attention_pipe(fp8, paged, tq, tk, tv, a, s);
     return launch_attention(fp8, paged, tq, tk, tv, a, s);
 }
 
@@ -430,6 +432,16 @@ bsa_status_t bsa_prefill_paged(bsa_tensor_t q, bsa_tensor_t out, const int32_t* 
 }
 
 const char* bsa_last_error(void) { return g_last_error.c_str(); }
+
+bsa_status_t bsa_selftest_wait_timeout(uint64_t limit_ns, cudaStream_t stream) {
+    if (limit_ns < 1000ull || limit_ns > 1000000000ull) return fail(BSA_ERR_INVALID_ARG, "limit_ns must be in [1e3, 1e9]");
+    bsa_status_t est;
+    unsigned* err = device_error_word(&est);
+    if (err == nullptr) return est;
+    const cudaError_t e = launch_wait_timeout_selftest(err, limit_ns, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "wait-timeout self-test launch");
+    return BSA_OK;
+}
 
 bsa_status_t bsa_check_device_error(cudaStream_t stream) {
     cudaError_t e = cudaStreamSynchronize(stream);

@@ -313,20 +313,24 @@ __global__ void __launch_bounds__(kThreads3, 2)
                     tmem_ld64(tS, rr);
                 tc_fence_before();
                 mbar_arrive(&bars->s_free);
-                float mx = -INFINITY;
-                if (j >= 0) {
+                // Masked scores become -inf here, outside the exponential loop: the causal part of
+                // the diagonal block, and all of a skipped block.
+                if (diag) {
+#pragma unroll
+                    for (int e = 0; e < BN; ++e)
+                        if (e > row) rr[e] = __float_as_uint(-INFINITY);
+                } else if (j < 0) {
+#pragma unroll
+                    for (int e = 0; e < BN; ++e) rr[e] = __float_as_uint(-INFINITY);
+                }
+                float mx;
+                {
                     float m8[8];
 #pragma unroll
                     for (int q = 0; q < 8; ++q) m8[q] = -INFINITY;
-                    if (!diag) {
 #pragma unroll
-                        for (int e = 0; e < BN; e += 2)
-                            m8[(e / 2) % 8] = max3f(m8[(e / 2) % 8], __uint_as_float(rr[e]), __uint_as_float(rr[e + 1]));
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < BN; ++e)
-                            if (e <= row) m8[e % 8] = fmaxf(m8[e % 8], __uint_as_float(rr[e]));
-                    }
+                    for (int e = 0; e < BN; e += 2)
+                        m8[(e / 2) % 8] = max3f(m8[(e / 2) % 8], __uint_as_float(rr[e]), __uint_as_float(rr[e + 1]));
                     mx = max3f(max3f(m8[0], m8[1], m8[2]), max3f(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
                 }
                 const float m_blk = mx * sl2;
@@ -345,10 +349,6 @@ __global__ void __launch_bounds__(kThreads3, 2)
                     float x0, x1;
                     unpack_f32x2(x, x0, x1);
                     float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
-                    if (diag || j < 0) {
-                        if (j < 0 || e > row) p0 = 0.f;
-                        if (j < 0 || e + 1 > row) p1 = 0.f;
-                    }
                     sum4[(e / 2) % 4] = add_f32x2(sum4[(e / 2) % 4], pack_f32x2(p0, p1));
                     rr[e] = __float_as_uint(p0);
                     rr[e + 1] = __float_as_uint(p1);

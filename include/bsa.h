@@ -154,6 +154,16 @@ bsa_status_t stem_score_noalloc(bsa_tensor_t q, bsa_tensor_t k, bsa_tensor_t v, 
                                 float softmax_scale, float* scores, int32_t nb_stride,
                                 cudaStream_t stream);
 
+/* Self-test of the failure path that every pipeline wait in the library shares.  It has no
+ * counterpart on the Stem pages; it exists so that the timeout handling can be checked on a
+ * real GPU without faulting or hanging it.  Launches one CTA on `stream` that allocates tensor
+ * memory, waits on an mbarrier that nothing ever arrives at, gives up after limit_ns
+ * nanoseconds (1e3 <= limit_ns <= 1e9, else BSA_ERR_INVALID_ARG and nothing is launched),
+ * records BSA_ERR_TIMEOUT in the current device's error word, frees its tensor memory and
+ * exits.  Returns BSA_OK once launched; a following bsa_check_device_error() returns
+ * BSA_ERR_TIMEOUT (and clears the word), and the context stays usable. */
+bsa_status_t bsa_selftest_wait_timeout(uint64_t limit_ns, cudaStream_t stream);
+
 /* Message of the last error returned on the calling thread ("" if none). */
 const char* bsa_last_error(void);
 

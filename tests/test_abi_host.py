@@ -92,4 +92,7 @@ def test_argument_errors_return_status(lib):
     sl = (ctypes.c_int32 * 1)(1024)
     assert lib.bsa_prefill_paged(_t(), _t(), P(1), sl, 1, _t(), _t(), 100, 32, P(1), 16, 8, 8, 128, 128, P(1), 9,
                                  P(1), 36, 0.0, None, None) == 2
+    # wait-timeout self-test: the limit must lie in [1 us, 1 s]
+    assert lib.bsa_selftest_wait_timeout(ctypes.c_uint64(0), None) == 1
+    assert lib.bsa_selftest_wait_timeout(ctypes.c_uint64(2_000_000_000), None) == 1
     assert lib.bsa_last_error().decode() != ""

@@ -18,7 +18,7 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
 
 
-@pytest.fixture(params=["ws", "ws2", "ws3", "serial"])
+@pytest.fixture(params=["ws", "ws2", "ws3", "ws4", "pipe", "serial"])
 def variant(request, monkeypatch):
     """Attention kernel: the persistent warp-specialised default, or the one-tile-per-CTA one."""
     monkeypatch.setenv("BSA_ATTN_VARIANT", request.param)
