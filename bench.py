@@ -149,7 +149,7 @@ def whole_job_tflops(eff_flop_per_rank: float, world: int, ms_per_step: float) -
 TRAFFIC_PER_TOKEN = {
     ("serial", "fp8", 64, 8, 128): (359.159296e6 + 487.020288e6) / 32768,
 }
-ATTN_DEFAULT = "serial"  # the kernel bsa_prefill runs when BSA_ATTN_VARIANT is unset
+ATTN_DEFAULT = "ws3"  # the kernel bsa_prefill runs when BSA_ATTN_VARIANT is unset
 
 
 def attn_traffic(fp8: bool, B: int, N: int, Hq: int, Hkv: int, D: int):

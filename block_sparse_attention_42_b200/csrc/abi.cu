@@ -141,19 +141,20 @@ bsa_status_t make_map(CUtensorMap* m, const void* base, int eb, uint64_t d, uint
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// Attention kernel.  Default: one query tile per CTA, two CTAs per SM (attn.cu), currently
-// the fastest on B200.  BSA_ATTN_VARIANT selects the persistent warp-specialised kernels
-// ("ws": 1 CTA/SM with two tiles in flight, "ws2"/"ws3": two pipelined CTAs per SM); all of
-// them compute the same result and the tests cross-check every one.
+// Attention kernel.  Default: ws3 (attn_ws3.cu: persistent, two pipelined CTAs per SM with a
+// TMA producer warp, an MMA warp and a softmax warpgroup; BF16 at d = 128 / block 128, whose
+// stages do not fit two CTAs per SM that way, runs ws2 with P in TMEM).  BSA_ATTN_VARIANT picks
+// another kernel: "serial" (attn.cu, one tile per CTA, no overlap inside a CTA), "pipe"
+// (attn_pipe.cu, one warpgroup that also issues), "ws4" (attn_ws4.cu, column-split softmax),
+// "ws2".  All compute the same result and the tests cross-check every one.
 cudaError_t launch_attn(bool fp8, bool paged, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                         const AttnArgs& a, cudaStream_t s) {
     const char* v = std::getenv("BSA_ATTN_VARIANT");
-    if (v && std::strcmp(v, "ws") == 0) return launch_attention_ws(fp8, paged, tq, tk, tv, a, s);
+    if (v && std::strcmp(v, "serial") == 0) return launch_attention(fp8, paged, tq, tk, tv, a, s);
     if (v && std::strcmp(v, "ws2") == 0) return launch_attention_ws2(fp8, paged, tq, tk, tv, a, s);
-    if (v && std::strcmp(v, "ws3") == 0) return launch_attention_ws3(fp8, paged, tq, tk, tv, a, s);
     if (v && std::strcmp(v, "ws4") == 0) return launch_attention_ws4(fp8, paged, tq, tk, tv, a, s);
     if (v && std::strcmp(v, "pipe") == 0) return launch_attention_pipe(fp8, paged, tq, tk, tv, a, s);
-    return launch_attention(fp8, paged, tq, tk, tv, a, s);
+    return launch_attention_ws3(fp8, paged, tq, tk, tv, a, s);
 }
 
 bsa_status_t attn_common_checks(const bsa_tensor_t& q, const bsa_tensor_t& k, const bsa_tensor_t& v,

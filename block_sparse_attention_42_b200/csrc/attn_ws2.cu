@@ -343,17 +343,22 @@ __global__ void __launch_bounds__(kThreads2, 2)
                 for (int hf = 0; hf < BN / 64; ++hf) {
                     uint32_t rr[64];
                     tmem_ld64(tS + hf * 64, rr);
+                    // Masked scores become -inf outside the exponential loop.
+                    if (diag) {
+#pragma unroll
+                        for (int e = 0; e < 64; ++e)
+                            if (hf * 64 + e > row) rr[e] = __float_as_uint(-INFINITY);
+                    } else if (j < 0) {
+#pragma unroll
+                        for (int e = 0; e < 64; ++e) rr[e] = __float_as_uint(-INFINITY);
+                    }
 #pragma unroll
                     for (int e = 0; e < 64; e += 2) {
                         const uint64_t x = fma_f32x2(pack_f32x2(__uint_as_float(rr[e]), __uint_as_float(rr[e + 1])),
                                                      sl2x2, negm);
                         float x0, x1;
                         unpack_f32x2(x, x0, x1);
-                        float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
-                        if (diag || j < 0) {
-                            if (j < 0 || hf * 64 + e > row) p0 = 0.f;
-                            if (j < 0 || hf * 64 + e + 1 > row) p1 = 0.f;
-                        }
+                        const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
                         sum4[(e / 2) % 4] = add_f32x2(sum4[(e / 2) % 4], pack_f32x2(p0, p1));
                         rr[e] = __float_as_uint(p0);
                         rr[e + 1] = __float_as_uint(p1);

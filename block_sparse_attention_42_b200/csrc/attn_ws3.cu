@@ -39,7 +39,12 @@ struct Cfg3 {
     static constexpr int QP = D * EB / 128;
     static constexpr int Q_BYTES = kBM3 * D * EB;
     static constexpr int KV_BYTES = BN * D * EB;
-    static constexpr int P_BYTES = kBM3 * BN * EB;
+    static constexpr int P_TILE = kBM3 * BN * EB;
+    // Two P buffers when four K/V stages still fit beside them: P(k) then waits for PV(k-2),
+    // not PV(k-1).  (With E4M3 at d = 128 the second buffer would cost the fourth stage, which
+    // measured slower on B200.)
+    static constexpr int NP = (kSmem3Limit - 3072 - Q_BYTES - 2 * P_TILE) / KV_BYTES >= 4 ? 2 : 1;
+    static constexpr int P_BYTES = NP * P_TILE;
     static constexpr int NS_FIT = (kSmem3Limit - 3072 - Q_BYTES - P_BYTES) / KV_BYTES;
     static constexpr int NS = NS_FIT > kMaxStages3 ? kMaxStages3 : NS_FIT;
     static constexpr int OFF_Q = 0;
@@ -64,7 +69,12 @@ constexpr float kPScale3 = FP8 ? 3.f : 0.f;
 
 struct Bars3 {
     uint64_t kv_full[kMaxStages3], kv_empty[kMaxStages3];
-    uint64_t q_full, q_empty, s_full, s_free, p_full, o_done, drain, tmem_free;
+    uint64_t q_full, q_empty, s_full, s_free, drain, tmem_free;
+    // Per P buffer: block g's P is written into buffer g % NP (p_full[g % NP]) and its PV
+    // completes o_done[g % NP].  With one barrier pair per buffer the softmax cannot complete a
+    // p_full phase twice before the MMA warp has consumed it: reusing the buffer first needs
+    // the PV issued after that phase.
+    uint64_t p_full[2], o_done[2];
     uint32_t tmem_slot;
     int abort_flag;
     int lst[kListChunk3];
@@ -91,8 +101,10 @@ __global__ void __launch_bounds__(kThreads3, 2)
         mbar_init(&bars->q_empty, 1);
         mbar_init(&bars->s_full, 1);
         mbar_init(&bars->s_free, 128);
-        mbar_init(&bars->p_full, 128);
-        mbar_init(&bars->o_done, 1);
+        mbar_init(&bars->p_full[0], 128);
+        mbar_init(&bars->p_full[1], 128);
+        mbar_init(&bars->o_done[0], 1);
+        mbar_init(&bars->o_done[1], 1);
         mbar_init(&bars->drain, 1);
         mbar_init(&bars->tmem_free, 128);
         bars->abort_flag = 0;
@@ -226,9 +238,10 @@ __global__ void __launch_bounds__(kThreads3, 2)
                 tc_commit(&bars->s_full);
                 return true;
             };
-            // O (+)= P V with V from ring index r and P from shared memory.
+            // O (+)= P V with V from ring index r and P from shared-memory buffer pc % NP.
             auto mma_pv = [&](uint32_t r, bool accumulate) -> bool {
-                if (!mbar_wait(&bars->p_full, pc & 1, abort_flag, a.err)) return false;
+                const uint32_t pb = pc % C::NP;
+                if (!mbar_wait(&bars->p_full[pb], (pc / C::NP) & 1, abort_flag, a.err)) return false;
                 ++pc;
                 const int st = r % C::NS;
                 if (!mbar_wait(&bars->kv_full[st], (r / C::NS) & 1, abort_flag, a.err)) return false;
@@ -237,7 +250,7 @@ __global__ void __launch_bounds__(kThreads3, 2)
 #pragma unroll
                 for (int kk = 0; kk < C::KSTEPS_O; ++kk) {
                     const uint32_t byte = kk * 32, pan = byte / 128, within = byte % 128;
-                    const uint64_t da = smem_desc_sw128(aP + pan * kBM3 * 128 + within, 16, 1024);
+                    const uint64_t da = smem_desc_sw128(aP + pb * C::P_TILE + pan * kBM3 * 128 + within, 16, 1024);
                     const uint64_t db = smem_desc_sw128(aV + kk * C::ROWS_PER_KSTEP * 128, BN * 128, 1024);
                     const uint32_t acc = (accumulate || kk > 0) ? 1u : 0u;
                     if constexpr (FP8)
@@ -246,7 +259,7 @@ __global__ void __launch_bounds__(kThreads3, 2)
                         mma_f16_ss(tmem + 128, da, db, idesc_o, acc);
                 }
                 tc_commit(&bars->kv_empty[st]);
-                tc_commit(&bars->o_done);
+                tc_commit(&bars->o_done[pb]);
                 return true;
             };
             while (ok && it.active) {
@@ -283,7 +296,13 @@ __global__ void __launch_bounds__(kThreads3, 2)
         const uint32_t tS = tmem + lane_base;
         uint8_t* sP = smem + C::OFF_P;
         const uint32_t tO = tmem + lane_base + 128;
-        uint32_t scount = 0, ocount = 0;
+        uint32_t scount = 0;
+        uint32_t g = 0;  // blocks this CTA's softmax has finished (all tiles)
+        // Waits until PV of global block gg is complete (it read P buffer gg % NP, wrote O).
+        auto wait_pv = [&](uint32_t gg) -> bool {
+            const bool w = mbar_wait(&bars->o_done[gg % C::NP], (gg / C::NP) & 1, abort_flag, a.err);
+            return __all_sync(0xFFFFFFFFu, w);
+        };
         const float sl2 = a.scale_log2;
         bool ok = true;
         TileIter it;
@@ -305,34 +324,50 @@ __global__ void __launch_bounds__(kThreads3, 2)
                 }
                 tc_fence_after();
                 const bool diag = (j == T.i);
-                // The whole S row in registers with one TMEM read; after it S may be overwritten.
+                // The S row in registers (E4M3: two 64-column TMEM reads, the second in flight
+                // while the max of the first half is taken); after them S may be overwritten.  Masked scores
+                // become -inf here, outside the exponential loop: the causal part of the diagonal
+                // block, and all of a skipped block.
                 uint32_t rr[BN];
-                if constexpr (BN == 128)
+                float m8[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) m8[q] = -INFINITY;
+                auto mask_max = [&](int base) {
+                    if (diag) {
+#pragma unroll
+                        for (int e = 0; e < 64; ++e)
+                            if (base + e > row) rr[base + e] = __float_as_uint(-INFINITY);
+                    } else if (j < 0) {
+#pragma unroll
+                        for (int e = 0; e < 64; ++e) rr[base + e] = __float_as_uint(-INFINITY);
+                    }
+#pragma unroll
+                    for (int e = 0; e < 64; e += 2)
+                        m8[(e / 2) % 8] =
+                            max3f(m8[(e / 2) % 8], __uint_as_float(rr[base + e]), __uint_as_float(rr[base + e + 1]));
+                };
+                if constexpr (BN == 128 && FP8) {
+                    tmem_ld64(tS, *reinterpret_cast<uint32_t(*)[64]>(rr));
+                    tmem_ld64_nowait(tS + 64, *reinterpret_cast<uint32_t(*)[64]>(rr + 64));
+                    mask_max(0);
+                    tmem_ld_wait64(*reinterpret_cast<uint32_t(*)[64]>(rr + 64));
+                    tc_fence_before();
+                    mbar_arrive(&bars->s_free);
+                    mask_max(64);
+                } else if constexpr (BN == 128) {
+                    // (BF16, d = 64: the overlapped form spills at this register budget)
                     tmem_ld128(tS, rr);
-                else
-                    tmem_ld64(tS, rr);
-                tc_fence_before();
-                mbar_arrive(&bars->s_free);
-                // Masked scores become -inf here, outside the exponential loop: the causal part of
-                // the diagonal block, and all of a skipped block.
-                if (diag) {
-#pragma unroll
-                    for (int e = 0; e < BN; ++e)
-                        if (e > row) rr[e] = __float_as_uint(-INFINITY);
-                } else if (j < 0) {
-#pragma unroll
-                    for (int e = 0; e < BN; ++e) rr[e] = __float_as_uint(-INFINITY);
+                    tc_fence_before();
+                    mbar_arrive(&bars->s_free);
+                    mask_max(0);
+                    mask_max(64);
+                } else {
+                    tmem_ld64(tS, *reinterpret_cast<uint32_t(*)[64]>(rr));
+                    tc_fence_before();
+                    mbar_arrive(&bars->s_free);
+                    mask_max(0);
                 }
-                float mx;
-                {
-                    float m8[8];
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) m8[q] = -INFINITY;
-#pragma unroll
-                    for (int e = 0; e < BN; e += 2)
-                        m8[(e / 2) % 8] = max3f(m8[(e / 2) % 8], __uint_as_float(rr[e]), __uint_as_float(rr[e + 1]));
-                    mx = max3f(max3f(m8[0], m8[1], m8[2]), max3f(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
-                }
+                const float mx = max3f(max3f(m8[0], m8[1], m8[2]), max3f(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
                 const float m_blk = mx * sl2;
                 float m_new = m_used;
                 if (m_blk > m_used + kRescale3<FP8>) m_new = m_blk;
@@ -353,17 +388,15 @@ __global__ void __launch_bounds__(kThreads3, 2)
                     rr[e] = __float_as_uint(p0);
                     rr[e + 1] = __float_as_uint(p1);
                 }
-                if (k > 0) {
-                    // PV(k-1) reads P (rewritten below) and writes O (maybe rescaled below).
-                    w_ok = mbar_wait(&bars->o_done, ocount & 1, abort_flag, a.err);
-                    ++ocount;
-                    w_ok = __all_sync(0xFFFFFFFFu, w_ok);
-                    if (!w_ok) {
+                // The PV that last read this P buffer must be complete.
+                if (g >= static_cast<uint32_t>(C::NP)) {
+                    if (!wait_pv(g - C::NP)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                 }
+                uint8_t* sPg = sP + (g % C::NP) * C::P_TILE;
                 // P -> shared memory in the 128-byte-swizzled K-major layout of the PV A operand.
                 if constexpr (FP8) {
 #pragma unroll
@@ -372,12 +405,11 @@ __global__ void __launch_bounds__(kThreads3, 2)
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
                             const int e = unit * 16 + q * 4;
-                            w4[q] = pack_e4m3x2(__uint_as_float(rr[e]), __uint_as_float(rr[e + 1])) |
-                                    (static_cast<uint32_t>(pack_e4m3x2(__uint_as_float(rr[e + 2]), __uint_as_float(rr[e + 3])))
-                                     << 16);
+                            w4[q] = pack_e4m3x4(__uint_as_float(rr[e]), __uint_as_float(rr[e + 1]),
+                                                __uint_as_float(rr[e + 2]), __uint_as_float(rr[e + 3]));
                         }
                         const int pan = unit / 8, cc = unit % 8;
-                        *reinterpret_cast<uint4*>(sP + pan * kBM3 * 128 + row * 128 + ((cc ^ (row & 7)) * 16)) =
+                        *reinterpret_cast<uint4*>(sPg + pan * kBM3 * 128 + row * 128 + ((cc ^ (row & 7)) * 16)) =
                             make_uint4(w4[0], w4[1], w4[2], w4[3]);
                     }
                 } else {
@@ -388,19 +420,34 @@ __global__ void __launch_bounds__(kThreads3, 2)
                         for (int q = 0; q < 4; ++q)
                             w4[q] = pack_bf16x2(__uint_as_float(rr[unit * 8 + 2 * q]), __uint_as_float(rr[unit * 8 + 2 * q + 1]));
                         const int pan = unit / 8, cc = unit % 8;
-                        *reinterpret_cast<uint4*>(sP + pan * kBM3 * 128 + row * 128 + ((cc ^ (row & 7)) * 16)) =
+                        *reinterpret_cast<uint4*>(sPg + pan * kBM3 * 128 + row * 128 + ((cc ^ (row & 7)) * 16)) =
                             make_uint4(w4[0], w4[1], w4[2], w4[3]);
                     }
                 }
                 fence_proxy_async_smem();
                 if (k > 0 && __any_sync(0xFFFFFFFFu, alpha != 1.f)) {
+                    // O *= alpha once PV(k-1) has finished accumulating into it, 64 TMEM columns at
+                    // a time (P is in shared memory, rr is free).
+                    if (C::NP > 1) {
+                        if (!wait_pv(g - 1)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                    }
+                    const uint64_t a2 = pack_f32x2(alpha, alpha);
 #pragma unroll 1
-                    for (int ch = 0; ch < D / 32; ++ch) {
-                        uint32_t ro[32];
-                        tmem_ld32(tO + ch * 32, ro);
+                    for (int ch = 0; ch < D / 64; ++ch) {
+                        uint32_t ro[64];
+                        tmem_ld64(tO + ch * 64, ro);
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) ro[e] = __float_as_uint(__uint_as_float(ro[e]) * alpha);
-                        tmem_st32(tO + ch * 32, ro);
+                        for (int e = 0; e < 64; e += 2) {
+                            float v0, v1;
+                            unpack_f32x2(mul_f32x2(pack_f32x2(__uint_as_float(ro[e]), __uint_as_float(ro[e + 1])), a2), v0, v1);
+                            ro[e] = __float_as_uint(v0);
+                            ro[e + 1] = __float_as_uint(v1);
+                        }
+                        tmem_st64(tO + ch * 64, ro);
                     }
                 }
                 float s0, s1, s2, s3, s4, s5, s6, s7;
@@ -413,13 +460,11 @@ __global__ void __launch_bounds__(kThreads3, 2)
                 m_used = m_new;
                 tmem_st_wait();
                 tc_fence_before();
-                mbar_arrive(&bars->p_full);
+                mbar_arrive(&bars->p_full[g % C::NP]);
+                ++g;
             }
             if (!ok) break;
-            bool w_ok = mbar_wait(&bars->o_done, ocount & 1, abort_flag, a.err);
-            ++ocount;
-            w_ok = __all_sync(0xFFFFFFFFu, w_ok);
-            if (!w_ok) break;
+            if (!wait_pv(g - 1)) break;
             tc_fence_after();
             const int t_row = T.i * a.block + row;
             const bool store = row < a.block && t_row < T.n_tok;

@@ -82,9 +82,5 @@ cudaError_t launch_wait_timeout_selftest(unsigned* err, uint64_t limit_ns, cudaS
 // One query tile per CTA, serial load -> S -> softmax -> PV per kept block (attn.cu).
 cudaError_t launch_attention(bool fp8, bool paged, const CUtensorMap& tq, const CUtensorMap& tk,
                              const CUtensorMap& tv, const AttnArgs& a, cudaStream_t s);
-// Persistent, warp-specialised: TMA producer, MMA issuer, two softmax warpgroups over two
-// query tiles in flight (attn_ws.cu).  The default.
-cudaError_t launch_attention_ws(bool fp8, bool paged, const CUtensorMap& tq, const CUtensorMap& tk,
-                                const CUtensorMap& tv, const AttnArgs& a, cudaStream_t s);
 
 }  // namespace bsa
