@@ -272,7 +272,17 @@ bsa_status_t stem_score(bsa_tensor_t q, bsa_tensor_t k, bsa_tensor_t v, int32_t 
     const int dt = q.dtype == BSA_BF16 ? 0 : (q.dtype == BSA_FP8_E4M3 ? 1 : 2);
     cudaError_t e = launch_pool(dt, targ(q), targ(k), targ(v), B, N, Hq, Hkv, d, block, qbar, kbar, vbar, stream);
     if (e != cudaSuccess) return cuda_fail(e, "pool launch");
-    e = launch_score(qbar, kbar, vbar, B, Hq, Hkv, nb, d, tau, metric, scores, nb_stride, stream);
+    // Score GEMM on the tensor cores (3xTF32, score_tc.cu); BSA_SCORE_VARIANT=simt selects the
+    // fp32 FMA kernel (score.cu), which computes the same scores to fp32 rounding.
+    const char* sv = std::getenv("BSA_SCORE_VARIANT");
+    if (sv && std::strcmp(sv, "simt") == 0) {
+        e = launch_score(qbar, kbar, vbar, B, Hq, Hkv, nb, d, tau, metric, scores, nb_stride, stream);
+    } else {
+        bsa_status_t est;
+        unsigned* err = device_error_word(&est);
+        if (err == nullptr) return est;
+        e = launch_score_tc(qbar, kbar, vbar, B, Hq, Hkv, nb, d, tau, metric, scores, nb_stride, err, stream);
+    }
     if (e != cudaSuccess) return cuda_fail(e, "score launch");
     return BSA_OK;
 }

@@ -27,6 +27,10 @@ cudaError_t launch_pool(int dtype, TensorArg q, TensorArg k, TensorArg v, int B,
                         int block, float* qbar, float* kbar, float* vbar, cudaStream_t s);
 
 // a2: block scores from pooled representations.
+// tcgen05 3xTF32 version of launch_score (score_tc.cu); err = device error word.
+cudaError_t launch_score_tc(const float* qbar, const float* kbar, const float* vbar, int B, int Hq, int Hkv, int nb,
+                            int d, float tau, int metric, float* scores, int nb_stride, unsigned* err,
+                            cudaStream_t s);
 cudaError_t launch_score(const float* qbar, const float* kbar, const float* vbar, int B, int Hq, int Hkv, int nb,
                          int d, float tau, int metric, float* scores, int nb_stride, cudaStream_t s);
 

@@ -152,6 +152,18 @@ __device__ __forceinline__ void mma_f16_ss(uint32_t d_tmem, uint64_t a_desc, uin
         : "memory");
 }
 
+// D[tmem] (+)= A[smem] * B[smem]^T, TF32 inputs (fp32 in shared memory; the low 13 mantissa
+// bits are not used), FP32 accumulate.
+__device__ __forceinline__ void mma_tf32_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // D[tmem] (+)= A[smem] * B[smem]^T, 8-bit float inputs (E4M3 here), FP32 accumulate.
 __device__ __forceinline__ void mma_f8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                           uint32_t accumulate) {
@@ -313,8 +325,9 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
     return d;
 }
 
-// Instruction descriptor (kind::f16 / kind::f8f6f4): FP32 accumulator, dense, no negation.
-// ab_format: kind::f16 -> 0 F16, 1 BF16; kind::f8f6f4 -> 0 E4M3, 1 E5M2.
+// Instruction descriptor (kind::f16 / kind::tf32 / kind::f8f6f4): FP32 accumulator, dense, no
+// negation.  ab_format: kind::f16 -> 0 F16, 1 BF16; kind::tf32 -> 2 TF32; kind::f8f6f4 -> 0 E4M3,
+// 1 E5M2.
 __host__ __device__ constexpr uint32_t make_idesc(int M, int N, uint32_t ab_format, bool a_mn_major,
                                                   bool b_mn_major) {
     return (1u << 4)                                  // D format: F32

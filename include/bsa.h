@@ -84,9 +84,11 @@ size_t bsa_score_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int32_t nb,
  *     scores[b, h, i, j] = tau * Qbar[b,h,i] . Kbar[b,h/G,j]  (+ ln vbar[b,h/G,j] for OAM)
  * with Qbar/Kbar the means of the block's token vectors (dequantised), vbar the mean L2 norm
  * of the block's value vectors, tau = softmax_scale.  scores is fp32 [B, Hq, nb_stride,
- * nb_stride] (nb_stride >= nb = ceil(N/block)); entries with j > i inside 64x64 tiles that
- * touch the diagonal are -inf, tiles wholly above it are not written.  ws: device workspace
- * of at least bsa_score_workspace_bytes() bytes, 256-byte aligned. */
+ * nb_stride] (nb_stride >= nb = ceil(N/block)); entries with j > i inside the 128x128 tiles
+ * that touch the diagonal are -inf, tiles wholly above it are not written.  The product runs
+ * on the tensor cores as three TF32 products (hi*hi + hi*lo + lo*hi of each operand's split),
+ * fp32-accurate.  ws: device workspace of at least bsa_score_workspace_bytes() bytes, 256-byte
+ * aligned. */
 bsa_status_t stem_score(bsa_tensor_t q, bsa_tensor_t k, bsa_tensor_t v, int32_t B, int32_t N,
                         int32_t Hq, int32_t Hkv, int32_t d, int32_t block, int32_t metric,
                         float softmax_scale, float* scores, int32_t nb_stride, void* ws,

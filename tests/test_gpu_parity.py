@@ -42,11 +42,22 @@ SCORE_CASES = [
     (inputs.gqa_8k(), 3000, "bf16", 0),        # ragged tail (3000 = 23 * 128 + 56)
     (inputs.gqa_8k(), 2048, "fp8", 0),
     (inputs.Workload("d64", 2, 4, 2, 1000, 64, 64, "bf16", 0.25, "stem", 7), None, "bf16", 0),
+    (inputs.gqa_8k(), 32768 + 300, "bf16", 0),  # nb = 259: several 128 x 128 score tiles + a ragged one
 ]
 
 
+@pytest.fixture(params=["tc", "simt"])
+def score_variant(request, monkeypatch):
+    """Score GEMM: tcgen05 3xTF32 (default) or the fp32 FMA kernel."""
+    if request.param == "simt":
+        monkeypatch.setenv("BSA_SCORE_VARIANT", "simt")
+    else:
+        monkeypatch.delenv("BSA_SCORE_VARIANT", raising=False)
+    return request.param
+
+
 @pytest.mark.parametrize("w,N,storage,metric", SCORE_CASES, ids=lambda x: getattr(x, "name", str(x)))
-def test_scores_match_oracle(orc, w, N, storage, metric):
+def test_scores_match_oracle(orc, score_variant, w, N, storage, metric):
     q, k, v, sq, sk, sv = _inputs(w, N, storage)
     B, N, Hq, d = q.shape
     tau = H.default_tau(d)
