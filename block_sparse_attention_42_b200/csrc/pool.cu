@@ -18,6 +18,7 @@ namespace bsa {
 namespace {
 
 constexpr int kPoolThreads = 256;
+constexpr int kBatch = 8;  // tokens whose loads each thread issues together
 
 template <int DT>
 struct Elem;
@@ -71,7 +72,7 @@ struct PoolArgs {
 };
 
 template <int DT>
-__global__ void __launch_bounds__(kPoolThreads) pool_kernel(const PoolArgs a) {
+__global__ void __launch_bounds__(kPoolThreads, 2) pool_kernel(const PoolArgs a) {
     constexpr int V = Elem<DT>::kVec;
     const int which = blockIdx.z;
     const TensorArg x = a.t[which];
@@ -102,29 +103,37 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const PoolArgs a) {
         double nacc = 0.0;
         const char* base = static_cast<const char*>(x.ptr);
         const int esz = DT == 0 ? 2 : (DT == 1 ? 1 : 4);
-        // Uniform trip count across the CTA so the warp shuffles below never diverge.
-        for (int tb = t_lo; tb < t_hi; tb += tg_count) {
-            const int t = tb + tg;
-            const bool ok = live && t < t_hi;
-            float f[V];
-            if (ok) {
-                const int64_t off = static_cast<int64_t>(b) * x.sb + static_cast<int64_t>(t) * x.st +
-                                    static_cast<int64_t>(h) * x.sh + c0;
-                const uint4 raw = __ldg(reinterpret_cast<const uint4*>(base + off * esz));
-                Elem<DT>::decode(raw, f);
-            } else {
+        // Tokens in batches of kBatch per thread: all of a batch's 16-byte loads are issued
+        // before any is consumed, so each thread keeps several HBM requests in flight.  The trip
+        // count is uniform across the CTA so the warp shuffles below never diverge.
+        for (int tb = t_lo; tb < t_hi; tb += tg_count * kBatch) {
+            uint4 raw[kBatch];
+            bool okb[kBatch];
 #pragma unroll
-                for (int e = 0; e < V; ++e) f[e] = 0.f;
+            for (int u = 0; u < kBatch; ++u) {
+                const int t = tb + u * tg_count + tg;
+                okb[u] = live && t < t_hi;
+                raw[u] = make_uint4(0u, 0u, 0u, 0u);
+                if (okb[u]) {
+                    const int64_t off = static_cast<int64_t>(b) * x.sb + static_cast<int64_t>(t) * x.st +
+                                        static_cast<int64_t>(h) * x.sh + c0;
+                    raw[u] = __ldg(reinterpret_cast<const uint4*>(base + off * esz));
+                }
             }
 #pragma unroll
-            for (int e = 0; e < V; ++e) acc[e] += static_cast<double>(f[e]);
-            if (is_v) {
-                double ss = 0.0;
+            for (int u = 0; u < kBatch; ++u) {
+                float f[V];
+                Elem<DT>::decode(raw[u], f);  // zero bits decode to +0 in every format
 #pragma unroll
-                for (int e = 0; e < V; ++e) ss += static_cast<double>(f[e]) * static_cast<double>(f[e]);
-                // Sum of squares over the head's d/V lanes (aligned power-of-two lane groups).
-                for (int o = 1; o < vec_per_head; o <<= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
-                if (ok) nacc += sqrt(ss);
+                for (int e = 0; e < V; ++e) acc[e] += static_cast<double>(f[e]);
+                if (is_v) {
+                    double ss = 0.0;
+#pragma unroll
+                    for (int e = 0; e < V; ++e) ss += static_cast<double>(f[e]) * static_cast<double>(f[e]);
+                    // Sum of squares over the head's d/V lanes (aligned power-of-two lane groups).
+                    for (int o = 1; o < vec_per_head; o <<= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
+                    if (okb[u]) nacc += sqrt(ss);
+                }
             }
         }
         if (vpt >= kPoolThreads) {
