@@ -81,7 +81,7 @@ def _check_lists_equal(rp_g, ci_g, rp_o, ci_o, nbs, Hq):
         assert np.array_equal(ci_g[b, :, :tot], ci_o[b, :, :tot])
 
 
-@pytest.mark.parametrize("density", [0.1, 0.25, 0.5, 1.0])
+@pytest.mark.parametrize("density", [0.1, 0.2, 0.25, 0.5, 0.8, 1.0])
 @pytest.mark.parametrize("decay", [0.5, 0.0])
 def test_select_bitexact_on_gpu_scores(orc, density, decay):
     w = inputs.gqa_8k()
@@ -173,6 +173,8 @@ ATTN_CASES = [
     ("d64-bs128", inputs.Workload("r", 2, 4, 1, 777, 64, 128, "bf16", 0.4, "normal", 12), None, "bf16", True),
     ("d128-bs64", inputs.Workload("r", 1, 2, 2, 1100, 128, 64, "bf16", 0.3, "stem", 13), None, "bf16", True),
     ("gqa-8k", inputs.gqa_8k(), None, "bf16", False),
+    ("sweep-32k-rho10", inputs.sweep_32k(0.1), None, "bf16", False),
+    ("sweep-32k-rho80", inputs.sweep_32k(0.8), None, "bf16", False),
 ]
 
 
