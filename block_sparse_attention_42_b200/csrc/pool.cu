@@ -37,18 +37,29 @@ struct Elem<0> {  // bf16
 template <>
 struct Elem<1> {  // e4m3
     static constexpr int kVec = 16;
+    // Exact decode with integer ops and one multiply (no conversion instructions): the code's
+    // 7 exponent/mantissa bits placed at fp32 bits 26..20 (sign at 31) read as 2^(e-127) *
+    // (1 + m/8), or as the denormal m/8 * 2^-126 when e = 0; times 2^120 that is the E4M3
+    // value (bias 7), subnormals included.  (Denormals are kept: no flush-to-zero here.)
     __device__ static void decode(const uint4& raw, float (&f)[16]) {
         const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[i] & 0xFFFFu), __NV_E4M3);
-            __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[i] >> 16), __NV_E4M3);
-            float2 a = __half22float2(*reinterpret_cast<__half2*>(&lo));
-            float2 b = __half22float2(*reinterpret_cast<__half2*>(&hi));
-            f[4 * i] = a.x;
-            f[4 * i + 1] = a.y;
-            f[4 * i + 2] = b.x;
-            f[4 * i + 3] = b.y;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const uint32_t b = (w[i] >> (8 * q)) & 0xFFu;
+                f[4 * i + q] = __uint_as_float(((b & 0x80u) << 24) | ((b & 0x7Fu) << 20)) * 0x1p120f;
+            }
+        }
+        // The NaN codes (x111_1111) would read as +-480 above: a word holding one has a byte
+        // whose low 7 bits + 1 carry into bit 7.
+        uint32_t nan_any = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) nan_any |= ((w[i] & 0x7F7F7F7Fu) + 0x01010101u) & 0x80808080u;
+        if (nan_any) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                if (((w[i / 4] >> (8 * (i % 4))) & 0x7Fu) == 0x7Fu) f[i] = __uint_as_float(0x7FC00000u);
         }
     }
 };
@@ -101,6 +112,13 @@ __global__ void __launch_bounds__(kPoolThreads, 2) pool_kernel(const PoolArgs a)
 #pragma unroll
         for (int e = 0; e < V; ++e) acc[e] = 0.0;
         double nacc = 0.0;
+        // E4M3: values are multiples of 2^-9 below 2^9, so any sum of up to 64 of them is exact
+        // in fp32; such partial sums are flushed into the fp64 sums every kFlush batches.
+        float facc[V];
+#pragma unroll
+        for (int e = 0; e < V; ++e) facc[e] = 0.f;
+        constexpr int kFlush = 64 / kBatch;
+        int nbatch = 0;
         const char* base = static_cast<const char*>(x.ptr);
         const int esz = DT == 0 ? 2 : (DT == 1 ? 1 : 4);
         // Tokens in batches of kBatch per thread: all of a batch's 16-byte loads are issued
@@ -124,17 +142,45 @@ __global__ void __launch_bounds__(kPoolThreads, 2) pool_kernel(const PoolArgs a)
             for (int u = 0; u < kBatch; ++u) {
                 float f[V];
                 Elem<DT>::decode(raw[u], f);  // zero bits decode to +0 in every format
+                if constexpr (DT == 1) {
 #pragma unroll
-                for (int e = 0; e < V; ++e) acc[e] += static_cast<double>(f[e]);
+                    for (int e = 0; e < V; ++e) facc[e] += f[e];
+                } else {
+#pragma unroll
+                    for (int e = 0; e < V; ++e) acc[e] += static_cast<double>(f[e]);
+                }
                 if (is_v) {
-                    double ss = 0.0;
+                    if constexpr (DT == 1) {
+                        // fp32 sum of squares (relative error ~1e-7 in the norm).
+                        float ss = 0.f;
 #pragma unroll
-                    for (int e = 0; e < V; ++e) ss += static_cast<double>(f[e]) * static_cast<double>(f[e]);
-                    // Sum of squares over the head's d/V lanes (aligned power-of-two lane groups).
-                    for (int o = 1; o < vec_per_head; o <<= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
-                    if (okb[u]) nacc += sqrt(ss);
+                        for (int e = 0; e < V; ++e) ss = fmaf(f[e], f[e], ss);
+                        for (int o = 1; o < vec_per_head; o <<= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
+                        if (okb[u]) nacc += static_cast<double>(sqrtf(ss));
+                    } else {
+                        double ss = 0.0;
+#pragma unroll
+                        for (int e = 0; e < V; ++e) ss += static_cast<double>(f[e]) * static_cast<double>(f[e]);
+                        // Sum of squares over the head's d/V lanes (aligned power-of-two lane groups).
+                        for (int o = 1; o < vec_per_head; o <<= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
+                        if (okb[u]) nacc += sqrt(ss);
+                    }
                 }
             }
+            if constexpr (DT == 1) {
+                if (++nbatch == kFlush) {
+#pragma unroll
+                    for (int e = 0; e < V; ++e) {
+                        acc[e] += static_cast<double>(facc[e]);
+                        facc[e] = 0.f;
+                    }
+                    nbatch = 0;
+                }
+            }
+        }
+        if constexpr (DT == 1) {
+#pragma unroll
+            for (int e = 0; e < V; ++e) acc[e] += static_cast<double>(facc[e]);
         }
         if (vpt >= kPoolThreads) {
             if (live) {

@@ -69,6 +69,27 @@ def test_scores_match_oracle(orc, score_variant, w, N, storage, metric):
     H.assert_scores_close(S[..., :nb, :nb], So, H.score_scale(qb, kb, vb, tau, metric), nb)
 
 
+def test_fp8_nan_code_pools_to_nan(orc):
+    """An E4M3 NaN code in Q makes that block's pooled row, hence its scores, NaN (as in the
+    oracle); every other score is unaffected."""
+    w = inputs.gqa_8k()
+    q, k, v, sq, sk, sv = _inputs(w, 2048, "fp8")
+    q.view(torch.uint8)[0, 700, 3, 17] = 0x7F  # token 700 -> query block 5, head 3
+    S = bsa.stem_score(q, k, v, w.block, q_scale=sq, k_scale=sk, v_scale=sv)
+    torch.cuda.synchronize()
+    qb, kb, vb = H.oracle_pool(orc, q, k, v, w.block, sq, sk, sv)
+    assert np.isnan(qb[0, 3, 5, 17])
+    So = orc.score(qb, kb, vb, H.default_tau(q.shape[-1]), 0)
+    nb = S.shape[-1]
+    g = S[0, 3, 5, :6].double().cpu().numpy()
+    assert np.all(np.isnan(g)) and np.all(np.isnan(So[0, 3, 5, :6]))
+    ok = np.ones(S.shape, bool)
+    ok[0, 3, 5, :] = False
+    Sg = S.double().cpu().numpy()
+    tri = np.broadcast_to(np.tril(np.ones((nb, nb), bool)), S.shape) & ok
+    assert np.all(np.isfinite(Sg[tri]) == np.isfinite(So[tri]))
+
+
 # ----------------------------------------------------------------------------- a3 + a4 select
 
 
