@@ -159,6 +159,20 @@ def attn_traffic(fp8: bool, B: int, N: int, Hq: int, Hkv: int, D: int):
     return None if per is None else per * B * N
 
 
+def mufu_roofline(res, device):
+    """exp2 throughput of bsa_prefill against the MUFU peak (bound 'alu')."""
+    props = torch.cuda.get_device_properties(device)
+    sms = props.multi_processor_count
+    mhz = (res.get("clocks") or {}).get("sm_mhz") or 1965.0
+    blk = res["w"].block
+    n_exp = float(res["kstar"]) * res["Hq"] * res["B"] * blk * blk  # kept blocks x block^2 per head
+    achieved = n_exp / (res["attn_ms_mean"] * 1e-3) / 1e12
+    peak = 16.0 * sms * mhz * 1e6 / 1e12
+    return {"bound": "alu", "unit": "Texp2/s", "achieved": achieved, "peak": peak, "frac": achieved / peak,
+            "peak_source": f"16 exp2/clk/SM (MUFU, measured) x {sms} SMs x {mhz:.0f} MHz sampled",
+            "kernel": "bsa_prefill"}
+
+
 def peaks():
     p = ROOT / "MEASURED_PEAKS.json"
     if p.exists():
@@ -493,6 +507,11 @@ def main():
                                         f"{' x2 (fp8/bf16 nominal ratio)' if fp8 else ''}",
                          "traffic": attn_traffic(fp8, res["B"], res["N"], res["Hq"], res["Hkv"], res["D"]),
                          "traffic_source": "ncu dram bytes of the fp8-32k capture, scaled by tokens"},
+            # The bound that binds for E4M3 attention: the exponentials.  Every kept 128-key
+            # block needs block x block exp2 per query row tile; the MUFU unit does 16 per clock
+            # per SM (measured with a throughput probe on this machine), so the peak is
+            # 16 x SMs x the median SM clock sampled during the timed steps.
+            "roofline_mufu": mufu_roofline(res, device),
             "gpu_launches": 5 * args.steps,
             "clocks": res["clocks"],
         }
