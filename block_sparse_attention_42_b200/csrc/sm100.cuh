@@ -288,18 +288,6 @@ __device__ __forceinline__ void mma_f8_ts(uint32_t d_tmem, uint32_t a_tmem, uint
         : "memory");
 }
 
-// Non-blocking probe of an mbarrier phase (no suspend).
-__device__ __forceinline__ uint32_t mbar_test(uint64_t* bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}\n"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok;
-}
 
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
@@ -418,40 +406,6 @@ __device__ __forceinline__ void exp2_poly_x2(float x0, float x1, float& y0, floa
     y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
 }
 
-// Packed half-precision helpers for the E4M3 softmax path.
-__device__ __forceinline__ uint32_t cvt_f16x2(float lo, float hi) {
-    uint32_t r;
-    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-    return r;
-}
-__device__ __forceinline__ uint32_t ex2_f16x2(uint32_t x) {
-    uint32_t r;
-    asm("ex2.approx.f16x2 %0, %1;" : "=r"(r) : "r"(x));
-    return r;
-}
-__device__ __forceinline__ uint32_t add_f16x2(uint32_t a, uint32_t b) {
-    uint32_t r;
-    asm("add.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
-    return r;
-}
-__device__ __forceinline__ uint32_t e4m3x2_from_f16x2(uint32_t x) {
-    uint16_t r;
-    asm("cvt.rn.satfinite.e4m3x2.f16x2 %0, %1;" : "=h"(r) : "r"(x));
-    return r;
-}
-// low 16 bits of a, then low 16 bits of b
-__device__ __forceinline__ uint32_t join16(uint32_t a, uint32_t b) {
-    uint32_t r;
-    asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(r) : "r"(a), "r"(b));
-    return r;
-}
-__device__ __forceinline__ float f16x2_hsum(uint32_t x) {
-    float lo, hi;
-    asm("{\n\t.reg .f16 l, h;\n\tmov.b32 {l, h}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, h;\n\t}\n"
-        : "=f"(lo), "=f"(hi)
-        : "r"(x));
-    return lo + hi;
-}
 
 // Two fp32 -> packed e4m3x2 (round to nearest even, saturate to the finite range).
 // Four floats -> four E4M3 bytes (a in the lowest byte), saturating, round to nearest even.
