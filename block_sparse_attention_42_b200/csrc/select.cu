@@ -203,8 +203,27 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_kernel(const float* __r
         int want = want_total;
         if (want_total > 0) {
             uint32_t prefix = 0, pmask = 0;
+            // High bytes shared by every candidate key (typical: the scores of a row have close
+            // exponents) are the same in the threshold; their passes would pick that byte with
+            // nothing above it, so they are skipped.
+            uint32_t kmn = 0xFFFFFFFFu, kmx = 0u;
+#pragma unroll
+            for (int r = 0; r < MAXPL; ++r) {
+                if (r * 32 < i + 1 && key[r] != 0u) {
+                    kmn = min(kmn, key[r]);
+                    kmx = max(kmx, key[r]);
+                }
+            }
+            kmn = __reduce_min_sync(0xFFFFFFFFu, kmn);
+            kmx = __reduce_max_sync(0xFFFFFFFFu, kmx);
+            int pass0 = 0;
+            while (pass0 < 4 && ((kmn ^ kmx) >> (24 - 8 * pass0)) == 0u) {
+                prefix |= kmx & (0xFFu << (24 - 8 * pass0));
+                pmask |= 0xFFu << (24 - 8 * pass0);
+                ++pass0;
+            }
 #pragma unroll 1
-            for (int pass = 0; pass < 4; ++pass) {
+            for (int pass = pass0; pass < 4; ++pass) {
                 const int shift = 24 - 8 * pass;
 #pragma unroll
                 for (int q = 0; q < 8; ++q) hist[lane * 8 + q] = 0;
