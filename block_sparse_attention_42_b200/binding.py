@@ -19,7 +19,7 @@ _lib = None
 BSA_BF16, BSA_FP8_E4M3, BSA_FP32 = 0, 1, 2
 BSA_METRIC_OAM, BSA_METRIC_SAM, BSA_METRIC_OAM_MUL = 0, 1, 2
 STATUS = {0: "BSA_OK", 1: "BSA_ERR_INVALID_ARG", 2: "BSA_ERR_UNSUPPORTED", 3: "BSA_ERR_CUDA",
-          4: "BSA_ERR_WORKSPACE", 5: "BSA_ERR_INVALID_LIST", 6: "BSA_ERR_TIMEOUT"}
+          4: "BSA_ERR_WORKSPACE", 5: "BSA_ERR_INVALID_LIST", 6: "BSA_ERR_TIMEOUT", 7: "BSA_ERR_INVALID_PAGE"}
 
 # Every symbol include/bsa.h declares.
 EXPORTS = ["bsa_tpd_budget", "bsa_score_workspace_bytes", "stem_score", "stem_select", "bsa_prefill",

@@ -19,6 +19,7 @@
 // drains its in-flight copies and MMAs with a bounded wait, frees its TMEM and exits.
 #include <cuda_bf16.h>
 
+#include "attn_tiles.cuh"
 #include "internal.h"
 #include "sm100.cuh"
 
@@ -133,6 +134,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV), aP = smem_u32(sP);
 
     bool kv_inflight = false, mma_inflight = false;
+    unsigned page_bad = 0;  // kDevErrInvalidPage if thread 0 met a page-table entry out of range
     uint32_t mma_parity = 0;
     if (tid == 0) {
         mbar_arrive_expect_tx(bar_q, C::Q_BYTES);
@@ -159,8 +161,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int pg = 0; pg < BN / 64; ++pg) {
                         const int lp = j * (BN / 64) + pg;
-                        const int phys = lp * 64 < n_tok ? a.page_table[static_cast<int64_t>(b) * a.max_pages + lp]
-                                                         : a.num_pages;  // past the end: zero fill
+                        const int phys = physical_page(a, b, lp, n_tok, page_bad);
                         tma_load_4d(sK + p * BN * 128 + pg * 64 * 128, &tk, bar_kv, p * C::PW, 0, hk, phys);
                         tma_load_4d(sV + p * BN * 128 + pg * 64 * 128, &tv, bar_kv, p * C::PW, 0, hk, phys);
                     }
@@ -328,6 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_wait(bar_o, mma_parity, &no_abort, a.err);
         }
     }
+    if (page_bad) atomicOr(a.err, page_bad);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();

@@ -25,6 +25,7 @@
 // issuing, drains its copies and MMAs with bounded waits, frees TMEM and exits.
 #include <cuda_bf16.h>
 
+#include "attn_tiles.cuh"
 #include "internal.h"
 #include "sm100.cuh"
 
@@ -155,7 +156,7 @@ __global__ void __launch_bounds__(kThreadsP, 1)
     // ---- thread 0's issue state
     uint32_t r_issued = 0;  // ring indices issued so far (loads)
     const uint32_t r_total = 2u * n_list;
-    bool bad = false;
+    unsigned bad = 0;  // kDevErr* bits found by thread 0's loads
     // Issues the loads of ring indices [r_issued, r_end).
     auto issue_loads = [&](uint32_t r_end) {
         if (r_end > r_total) r_end = r_total;
@@ -163,7 +164,7 @@ __global__ void __launch_bounds__(kThreadsP, 1)
             const int n = static_cast<int>(r_issued >> 1);
             int j = __ldg(gl + n);
             if (j < 0 || j > i) {  // out of the causal range: flagged; the softmax zeroes it
-                bad = true;
+                bad |= kDevErrInvalidList;
                 j = 0;
             }
             const int st = r_issued % C::NS;
@@ -177,8 +178,7 @@ __global__ void __launch_bounds__(kThreadsP, 1)
 #pragma unroll
                     for (int pg = 0; pg < BN / 64; ++pg) {
                         const int lp = j * (BN / 64) + pg;
-                        const int phys = lp * 64 < n_tok ? __ldg(a.page_table + static_cast<int64_t>(b) * a.max_pages + lp)
-                                                         : a.num_pages;  // past the end: zero fill
+                        const int phys = physical_page(a, b, lp, n_tok, bad);
                         tma_load_4d(dst + p * BN * 128 + pg * 64 * 128, map, fb, p * C::PW, 0, hk, phys);
                     }
                 } else {
@@ -422,7 +422,7 @@ __global__ void __launch_bounds__(kThreadsP, 1)
         tc_commit(&bars->drain);
         mbar_wait(&bars->drain, 0, &no_abort, a.err);
     }
-    if (tid == 0 && bad) atomicOr(a.err, kDevErrInvalidList);
+    if (tid == 0 && bad) atomicOr(a.err, bad);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();

@@ -42,6 +42,19 @@ __device__ __forceinline__ Tile decode_tile(const AttnArgs& a, int t) {
     return T;
 }
 
+// Physical page of logical page lp (tokens 64*lp ...) of sequence b for a paged K/V load:
+// num_pages (a box the TMA reads as zeros) past the end of the sequence; an entry outside
+// [0, num_pages) is recorded in `bad` (kDevErrInvalidPage) and read as zeros too.
+__device__ __forceinline__ int physical_page(const AttnArgs& a, int b, int lp, int n_tok, unsigned& bad) {
+    if (lp * 64 >= n_tok) return a.num_pages;
+    const int phys = __ldg(a.page_table + static_cast<int64_t>(b) * a.max_pages + lp);
+    if (phys < 0 || phys >= a.num_pages) {
+        bad |= kDevErrInvalidPage;
+        return a.num_pages;
+    }
+    return phys;
+}
+
 // List entry n of the tile; -1 if out of [0, i] (skipped block: scores all -inf).
 __device__ __forceinline__ int list_entry(const AttnArgs& a, const Tile& T, int n) {
     const int j = __ldg(a.col_idx + (static_cast<int64_t>(T.b) * a.Hq + T.h) * a.max_k + T.l_begin + n);

@@ -179,7 +179,7 @@ __global__ void __launch_bounds__(kThreads4, 2)
                     for (int k = kb; ok && k < kend; ++k) {
                         int j = bars->lst[k - kb];
                         if (j < 0) {
-                            bad = 1;
+                            bad |= kDevErrInvalidList;
                             j = 0;
                         }
                         for (int v = 0; ok && v < 2; ++v) {
@@ -196,10 +196,7 @@ __global__ void __launch_bounds__(kThreads4, 2)
 #pragma unroll
                                     for (int pg = 0; pg < BN / 64; ++pg) {
                                         const int lp = j * (BN / 64) + pg;
-                                        const int phys =
-                                            lp * 64 < T.n_tok
-                                                ? __ldg(a.page_table + static_cast<int64_t>(T.b) * a.max_pages + lp)
-                                                : a.num_pages;  // past the end of the sequence: zeros
+                                        const int phys = physical_page(a, T.b, lp, T.n_tok, bad);
                                         tma_load_4d(dst + p * BN * 128 + pg * 64 * 128, map, fb, p * C::PW, 0, T.hk, phys);
                                     }
                                 } else {
@@ -215,7 +212,7 @@ __global__ void __launch_bounds__(kThreads4, 2)
             it.next(a);
         }
         if (lane == 0) {
-            if (bad) atomicOr(a.err, kDevErrInvalidList);
+            if (bad) atomicOr(a.err, bad);
             // Every issued copy must land before the CTA's shared memory goes away.
             volatile int no_abort = 0;
             for (uint32_t r = ring > C::NS ? ring - C::NS : 0; r < ring; ++r)

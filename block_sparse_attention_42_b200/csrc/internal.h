@@ -11,6 +11,7 @@ namespace bsa {
 // Device error word bits (read back by bsa_check_device_error).
 constexpr unsigned kDevErrInvalidList = 1u;
 constexpr unsigned kDevErrTimeout = 2u;
+constexpr unsigned kDevErrInvalidPage = 4u;
 
 constexpr int kMaxBatch = 256;     // sequences per call
 constexpr int kMaxBlocks = 2048;   // query blocks per sequence

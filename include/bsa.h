@@ -23,8 +23,8 @@
  *   - Calls are asynchronous on `stream`.  Argument errors are returned synchronously, with
  *     nothing launched, and the message is available from bsa_last_error().  A failed launch
  *     returns BSA_ERR_CUDA.  Errors found by kernels while running (an out-of-range list
- *     entry, an internal wait that ran out of time) are recorded in a per-device error word
- *     that bsa_check_device_error() reads.
+ *     entry, an out-of-range page-table entry, an internal wait that ran out of time) are
+ *     recorded in a per-device error word that bsa_check_device_error() reads.
  *   - Tensors are described by bsa_tensor_t: element strides of batch, token and head; the
  *     feature (head_dim) dimension is contiguous; the base pointer and every stride must be
  *     16-byte aligned in bytes.  `scale` is the per-tensor dequantisation scale of FP8 data
@@ -51,7 +51,8 @@ typedef enum {
     BSA_ERR_CUDA = 3,         /* a CUDA runtime/driver call or a launch failed */
     BSA_ERR_WORKSPACE = 4,    /* the workspace is missing or too small */
     BSA_ERR_INVALID_LIST = 5, /* (device) a list entry was outside [0, query block] */
-    BSA_ERR_TIMEOUT = 6       /* (device) an internal pipeline wait ran out of time */
+    BSA_ERR_TIMEOUT = 6,      /* (device) an internal pipeline wait ran out of time */
+    BSA_ERR_INVALID_PAGE = 7  /* (device) a page-table entry was outside [0, num_pages) */
 } bsa_status_t;
 
 typedef enum { BSA_BF16 = 0, BSA_FP8_E4M3 = 1, BSA_FP32 = 2 } bsa_dtype_t;
@@ -123,7 +124,9 @@ bsa_status_t bsa_prefill(bsa_tensor_t q, bsa_tensor_t k, bsa_tensor_t v, bsa_ten
  * length.  k_cache/v_cache are page pools [num_pages, page_size, Hkv, d] described with
  * stride_b = page stride and stride_t = slot stride; page_table [B, max_pages] int32 maps a
  * sequence's logical page p (tokens p*page_size ...) to a physical page.  page_size must be
- * 64 and divide `block`.  Lists and lse ([B, Hq, max_b N_b]) as in bsa_prefill. */
+ * 64 and divide `block`.  Lists and lse ([B, Hq, max_b N_b]) as in bsa_prefill.  A page entry
+ * outside [0, num_pages) for a page that holds tokens of the sequence is read as zeros and
+ * recorded (bsa_check_device_error then returns BSA_ERR_INVALID_PAGE). */
 bsa_status_t bsa_prefill_paged(bsa_tensor_t q, bsa_tensor_t out, const int32_t* cu_seqlens,
                                const int32_t* seqlens_host, int32_t B, bsa_tensor_t k_cache,
                                bsa_tensor_t v_cache, int32_t num_pages, int32_t page_size,
@@ -170,7 +173,8 @@ bsa_status_t bsa_selftest_wait_timeout(uint64_t limit_ns, cudaStream_t stream);
 const char* bsa_last_error(void);
 
 /* Synchronises `stream`, then reads and clears the current device's error word: returns
- * BSA_ERR_INVALID_LIST or BSA_ERR_TIMEOUT if a kernel recorded one, else BSA_OK. */
+ * BSA_ERR_TIMEOUT, BSA_ERR_INVALID_LIST or BSA_ERR_INVALID_PAGE if a kernel recorded one (in
+ * that order of precedence), else BSA_OK. */
 bsa_status_t bsa_check_device_error(cudaStream_t stream);
 
 #ifdef __cplusplus

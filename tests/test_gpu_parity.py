@@ -283,6 +283,35 @@ def test_paged_equals_contiguous(variant):
         assert torch.equal(outp[d["cu_seqlens"][b]:d["cu_seqlens"][b + 1]], ref[0]), b
 
 
+def test_invalid_page_entry_is_flagged(variant):
+    """A page-table entry outside [0, num_pages) for a page inside its sequence is read as zeros
+    and reported as BSA_ERR_INVALID_PAGE (no out-of-range access)."""
+    w = inputs.paged_varlen(seqlens=(1000, 300))
+    d = inputs.make_paged(w, device=DEV)
+    nbp = [(n + 127) // 128 for n in d["seqlens"]]
+    nbs = max(nbp)
+    S = torch.full((len(nbp), w.Hq, nbs, nbs), float("nan"), device=DEV)
+    for b in range(len(nbp)):
+        qb = d["q"][d["cu_seqlens"][b]:d["cu_seqlens"][b + 1]].unsqueeze(0)
+        bsa.stem_score(qb, d["k_seq"][b].unsqueeze(0), d["v_seq"][b].unsqueeze(0), 128, scores=S[b:b + 1],
+                       nb_stride=nbs)
+    rp, ci = bsa.stem_select(S, nbp, 0.25)
+    cu = d["cu_seqlens"].to(DEV)
+    bsa.bsa_check_device_error()
+    pt = d["page_table"].clone()
+    pt[0, 3] = d["num_pages"] + 7  # tokens 192..255 of sequence 0 (the diagonal block of query block 1)
+    bsa.bsa_prefill_paged(d["q"], cu, d["seqlens"], d["k_cache"], d["v_cache"], pt, 128, rp, ci)
+    with pytest.raises(bsa.BsaError) as ei:
+        bsa.bsa_check_device_error()
+    assert ei.value.status == 7
+    pt[0, 3] = -2
+    bsa.bsa_prefill_paged(d["q"], cu, d["seqlens"], d["k_cache"], d["v_cache"], pt, 128, rp, ci)
+    with pytest.raises(bsa.BsaError) as ei:
+        bsa.bsa_check_device_error()
+    assert ei.value.status == 7
+    bsa.bsa_check_device_error()  # cleared
+
+
 def test_invalid_list_entry_is_flagged(variant):
     w = inputs.Workload("bad", 1, 2, 1, 512, 128, 128, "bf16", 0.5, "normal", 17)
     q, k, v, *_ = _inputs(w)
