@@ -45,6 +45,9 @@ def parse():
     p.add_argument("--density", type=float, default=0.25)
     p.add_argument("--no-dense", action="store_true", help="skip the density-1 ideal-line measurement")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--e2e-split", type=int, default=1,
+                   help="query-head chunks per KV-head group in the pipelined end-to-end step (1 measured "
+                        "fastest at fp8-128k: 56.0 ms vs 57.3 / 62.3 for 2 / 4)")
     p.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
     return p.parse_args()
 
@@ -271,63 +274,74 @@ def run_ours(args, rank, world, device):
         del dense_out, dense_ci
 
     # End to end through the public API with host buffers: H2D of Q/K/V from pinned memory,
-    # the step, D2H of the output, all inside the timed region.  The step is pipelined over the
-    # Hkv head groups (each group's heads are an independent problem with its own lists): one
-    # stream uploads group g+1 while another runs score -> select -> prefill of group g and a
-    # third downloads group g-1's output, so the PCIe transfers (both directions) overlap the
-    # kernels.  Host and device buffers are per group and contiguous.
+    # the step, D2H of the output, all inside the timed region.  The step is pipelined over
+    # chunks of query heads (e2e_split chunks per KV-head group; every head is an independent
+    # problem with its own lists): one stream uploads chunk c+1 (with its group's K/V the first
+    # time), another runs score -> select -> prefill of chunk c and a third downloads chunk
+    # c-1's output, so the PCIe transfers (both directions) overlap the kernels.  Host and
+    # device buffers are per chunk (K/V per group) and contiguous.
     if not args.no_e2e:
         G = Hkv
         gq = Hq // G
-        sl = [slice(g * gq, (g + 1) * gq) for g in range(G)]
-        hq = [q[:, :, sl[g]].contiguous().cpu().pin_memory() for g in range(G)]
+        F = max(1, min(args.e2e_split, gq))
+        while gq % F:
+            F -= 1
+        cq = gq // F                       # query heads per chunk
+        NC = G * F                          # chunks: F per KV-head group, K/V uploaded with the first
+        slq = [slice(c * cq, (c + 1) * cq) for c in range(NC)]
+        hq = [q[:, :, slq[c]].contiguous().cpu().pin_memory() for c in range(NC)]
         hk = [k[:, :, g:g + 1].contiguous().cpu().pin_memory() for g in range(G)]
         hv = [v[:, :, g:g + 1].contiguous().cpu().pin_memory() for g in range(G)]
-        hout = [torch.empty((B, N, gq, D), dtype=out.dtype, pin_memory=True) for _ in range(G)]
+        hout = [torch.empty((B, N, cq, D), dtype=out.dtype, pin_memory=True) for _ in range(NC)]
         dq = [torch.empty_like(x, device=device) for x in hq]
         dk = [torch.empty_like(x, device=device) for x in hk]
         dv = [torch.empty_like(x, device=device) for x in hv]
-        dout = [torch.empty((B, N, gq, D), dtype=out.dtype, device=device) for _ in range(G)]
-        g_scores = torch.empty(B, gq, nb, nb, dtype=torch.float32, device=device)
-        g_ws = torch.empty(bsa.bsa_score_workspace_bytes(B, gq, 1, nb, D), dtype=torch.uint8, device=device)
+        dout = [torch.empty((B, N, cq, D), dtype=out.dtype, device=device) for _ in range(NC)]
+        g_scores = torch.empty(B, cq, nb, nb, dtype=torch.float32, device=device)
+        g_ws = torch.empty(bsa.bsa_score_workspace_bytes(B, cq, 1, nb, D), dtype=torch.uint8, device=device)
         g_rp = torch.empty(B, nb + 1, dtype=torch.int32, device=device)
-        g_ci = torch.empty(B, gq, kstar, dtype=torch.int32, device=device)
+        g_ci = torch.empty(B, cq, kstar, dtype=torch.int32, device=device)
         s_in, s_cmp, s_out = (torch.cuda.Stream(device) for _ in range(3))
-        ev_in = [torch.cuda.Event() for _ in range(G)]
-        ev_cmp = [torch.cuda.Event() for _ in range(G)]
-        ev_out = [torch.cuda.Event() for _ in range(G)]
+        ev_in = [torch.cuda.Event() for _ in range(NC)]
+        ev_cmp = [torch.cuda.Event() for _ in range(NC)]
+        ev_out = [torch.cuda.Event() for _ in range(NC)]
         started = [False]
 
         def e2e_step():
-            for g in range(G):
+            for c in range(NC):
+                g = c // F
                 with torch.cuda.stream(s_in):
                     if started[0]:
-                        s_in.wait_event(ev_cmp[g])  # the previous step's kernels of group g are done with dq/dk/dv
-                    dq[g].copy_(hq[g], non_blocking=True)
-                    dk[g].copy_(hk[g], non_blocking=True)
-                    dv[g].copy_(hv[g], non_blocking=True)
-                    ev_in[g].record(s_in)
-            for g in range(G):
+                        s_in.wait_event(ev_cmp[c])  # the previous step's kernels of chunk c are done with its inputs
+                        if c % F == 0:
+                            s_in.wait_event(ev_cmp[c + F - 1])  # ... and every chunk of group g with its K/V
+                    dq[c].copy_(hq[c], non_blocking=True)
+                    if c % F == 0:
+                        dk[g].copy_(hk[g], non_blocking=True)
+                        dv[g].copy_(hv[g], non_blocking=True)
+                    ev_in[c].record(s_in)
+            for c in range(NC):
+                g = c // F
                 with torch.cuda.stream(s_cmp):
-                    s_cmp.wait_event(ev_in[g])
+                    s_cmp.wait_event(ev_in[c])
                     if started[0]:
-                        s_cmp.wait_event(ev_out[g])  # the previous step's download of dout[g] is done
-                    bsa.stem_score(dq[g], dk[g], dv[g], w.block, scores=g_scores, workspace=g_ws, **scale_kw)
+                        s_cmp.wait_event(ev_out[c])  # the previous step's download of dout[c] is done
+                    bsa.stem_score(dq[c], dk[g], dv[g], w.block, scores=g_scores, workspace=g_ws, **scale_kw)
                     bsa.stem_select(g_scores, [nb] * B, w.density, 0.5, row_ptr=g_rp, col_idx=g_ci, max_k=kstar)
-                    bsa.bsa_prefill(dq[g], dk[g], dv[g], w.block, g_rp, g_ci, out=dout[g], **scale_kw)
-                    ev_cmp[g].record(s_cmp)
+                    bsa.bsa_prefill(dq[c], dk[g], dv[g], w.block, g_rp, g_ci, out=dout[c], **scale_kw)
+                    ev_cmp[c].record(s_cmp)
                 with torch.cuda.stream(s_out):
-                    s_out.wait_event(ev_cmp[g])
-                    hout[g].copy_(dout[g], non_blocking=True)
-                    ev_out[g].record(s_out)
+                    s_out.wait_event(ev_cmp[c])
+                    hout[c].copy_(dout[c], non_blocking=True)
+                    ev_out[c].record(s_out)
             started[0] = True
 
         main = torch.cuda.current_stream(device)
         e2e_step()
         torch.cuda.synchronize(device)
         # the pipelined output equals the full-size call's
-        for g in (0, G - 1):
-            assert torch.equal(hout[g], out[:, :, sl[g]].cpu()), "pipelined e2e output differs from the full call"
+        for c in (0, NC - 1):
+            assert torch.equal(hout[c], out[:, :, slq[c]].cpu()), "pipelined e2e output differs from the full call"
         n_e2e = max(1, min(args.steps, 3))
         if world > 1:
             torch.distributed.barrier()
@@ -344,7 +358,7 @@ def run_ours(args, rank, world, device):
         res["e2e_ms"] = reduce_max(e0.elapsed_time(e1) / n_e2e, world, device)
         res["h2d_bytes"] = sum(x.numel() * x.element_size() for x in (q, k, v))
         res["d2h_bytes"] = out.numel() * out.element_size()
-        res["e2e_pipeline"] = f"{G} head groups, H2D / kernels / D2H on three streams"
+        res["e2e_pipeline"] = f"{NC} chunks ({G} KV-head groups x {F}), H2D / kernels / D2H on three streams"
         del hq, hk, hv, hout, dq, dk, dv, dout, g_scores, g_ws, g_rp, g_ci
 
     res["cpu"] = None
