@@ -134,7 +134,7 @@ def stem_score(q, k, v, block: int, metric: int = BSA_METRIC_OAM, softmax_scale:
 
 def stem_score_noalloc(q, k, v, block: int, metric: int = BSA_METRIC_OAM, softmax_scale: float = 0.0,
                        scores=None, nb_stride: int | None = None, q_scale=1.0, k_scale=1.0, v_scale=1.0):
-    """stem_score with the library's fixed 16 MiB scratch instead of a workspace (for callers
+    """stem_score with the library's fixed 32 MiB scratch instead of a workspace (for callers
     that cannot allocate device memory).  Calls that overlap on the GPU race on that scratch."""
     B, N, Hq, d = q.shape
     Hkv = k.shape[2]

@@ -132,7 +132,10 @@ bsa_status_t make_map(CUtensorMap* m, const void* base, int eb, uint64_t d, uint
                                    static_cast<cuuint64_t>(s_outer) * eb};
     const cuuint32_t box[4] = {static_cast<cuuint32_t>(128 / eb), box_rows, 1, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
-    CUresult r = fn(m, eb == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 4,
+    const CUtensorMapDataType dt = eb == 4   ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                   : eb == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                             : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+    CUresult r = fn(m, dt, 4,
                     const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(BSA_ERR_INVALID_ARG, "%s: cuTensorMapEncodeTiled failed (%d)", name, (int)r);
@@ -241,8 +244,8 @@ int64_t bsa_tpd_budget(int32_t nb, double density, double tpd_decay, int32_t* k_
 
 size_t bsa_score_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int32_t nb, int32_t d) {
     if (B < 1 || Hq < 1 || Hkv < 1 || nb < 1 || d < 1) return 0;
-    return align256(sizeof(float) * size_t(B) * Hq * nb * d) + align256(sizeof(float) * size_t(B) * Hkv * nb * d) +
-           align256(sizeof(float) * size_t(B) * Hkv * nb);
+    return 2 * align256(sizeof(float) * size_t(B) * Hq * nb * d) +
+           2 * align256(sizeof(float) * size_t(B) * Hkv * nb * d) + align256(sizeof(float) * size_t(B) * Hkv * nb);
 }
 
 bsa_status_t stem_score(bsa_tensor_t q, bsa_tensor_t k, bsa_tensor_t v, int32_t B, int32_t N, int32_t Hq,
@@ -264,24 +267,38 @@ bsa_status_t stem_score(bsa_tensor_t q, bsa_tensor_t k, bsa_tensor_t v, int32_t 
     const size_t need = bsa_score_workspace_bytes(B, Hq, Hkv, nb, d);
     if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u))
         return fail(BSA_ERR_WORKSPACE, "workspace must be >= %zu bytes and 256-byte aligned", need);
-    float* qbar = static_cast<float*>(ws);
-    float* kbar = reinterpret_cast<float*>(static_cast<char*>(ws) + align256(sizeof(float) * size_t(B) * Hq * nb * d));
-    float* vbar = reinterpret_cast<float*>(reinterpret_cast<char*>(kbar) +
-                                           align256(sizeof(float) * size_t(B) * Hkv * nb * d));
+    // Workspace: [qhi | qlo | khi | klo | vbar], each part 256-byte aligned.
+    const size_t qbytes = align256(sizeof(float) * size_t(B) * Hq * nb * d);
+    const size_t kbytes = align256(sizeof(float) * size_t(B) * Hkv * nb * d);
+    char* w = static_cast<char*>(ws);
+    float* qhi = reinterpret_cast<float*>(w);
+    float* qlo = reinterpret_cast<float*>(w + qbytes);
+    float* khi = reinterpret_cast<float*>(w + 2 * qbytes);
+    float* klo = reinterpret_cast<float*>(w + 2 * qbytes + kbytes);
+    float* vbar = reinterpret_cast<float*>(w + 2 * qbytes + 2 * kbytes);
     const float tau = softmax_scale > 0.f ? softmax_scale : 1.f / std::sqrt(static_cast<float>(d));
     const int dt = q.dtype == BSA_BF16 ? 0 : (q.dtype == BSA_FP8_E4M3 ? 1 : 2);
-    cudaError_t e = launch_pool(dt, targ(q), targ(k), targ(v), B, N, Hq, Hkv, d, block, qbar, kbar, vbar, stream);
+    cudaError_t e =
+        launch_pool(dt, targ(q), targ(k), targ(v), B, N, Hq, Hkv, d, block, qhi, qlo, khi, klo, vbar, stream);
     if (e != cudaSuccess) return cuda_fail(e, "pool launch");
     // Score GEMM on the tensor cores (3xTF32, score_tc.cu); BSA_SCORE_VARIANT=simt selects the
     // fp32 FMA kernel (score.cu), which computes the same scores to fp32 rounding.
     const char* sv = std::getenv("BSA_SCORE_VARIANT");
     if (sv && std::strcmp(sv, "simt") == 0) {
-        e = launch_score(qbar, kbar, vbar, B, Hq, Hkv, nb, d, tau, metric, scores, nb_stride, stream);
+        e = launch_score(qhi, qlo, khi, klo, vbar, B, Hq, Hkv, nb, d, tau, metric, scores, nb_stride, stream);
     } else {
         bsa_status_t est;
         unsigned* err = device_error_word(&est);
         if (err == nullptr) return est;
-        e = launch_score_tc(qbar, kbar, vbar, B, Hq, Hkv, nb, d, tau, metric, scores, nb_stride, err, stream);
+        CUtensorMap mqh, mql, mkh, mkl;
+        const int64_t ro = d, qh = int64_t(nb) * d, kh = int64_t(nb) * d;
+        if ((st = make_map(&mqh, qhi, 4, d, nb, Hq, B, ro, qh, qh * Hq, 128, "qhi")) ||
+            (st = make_map(&mql, qlo, 4, d, nb, Hq, B, ro, qh, qh * Hq, 128, "qlo")) ||
+            (st = make_map(&mkh, khi, 4, d, nb, Hkv, B, ro, kh, kh * Hkv, 128, "khi")) ||
+            (st = make_map(&mkl, klo, 4, d, nb, Hkv, B, ro, kh, kh * Hkv, 128, "klo")))
+            return st;
+        e = launch_score_tc(mqh, mql, mkh, mkl, vbar, B, Hq, Hkv, nb, d, tau, metric, scores, nb_stride, err,
+                            stream);
     }
     if (e != cudaSuccess) return cuda_fail(e, "score launch");
     return BSA_OK;

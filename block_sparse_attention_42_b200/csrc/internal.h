@@ -22,18 +22,22 @@ struct TensorArg {
     float scale;
 };
 
-// a1: pooled block representations.  Writes qbar [B,Hq,nb,d], kbar [B,Hkv,nb,d] and
-// vbar [B,Hkv,nb] (fp32).  dtype: 0 bf16, 1 e4m3, 2 fp32.
+// a1: pooled block representations.  Writes the Q means [B,Hq,nb,d] as qbar = qhi + qlo (qhi
+// exact in TF32, qlo the fp32 remainder), the K means [B,Hkv,nb,d] as khi + klo, and the mean
+// V norms vbar [B,Hkv,nb] (fp32).  dtype: 0 bf16, 1 e4m3, 2 fp32.
 cudaError_t launch_pool(int dtype, TensorArg q, TensorArg k, TensorArg v, int B, int N, int Hq, int Hkv, int d,
-                        int block, float* qbar, float* kbar, float* vbar, cudaStream_t s);
+                        int block, float* qhi, float* qlo, float* khi, float* klo, float* vbar, cudaStream_t s);
 
 // a2: block scores from pooled representations.
-// tcgen05 3xTF32 version of launch_score (score_tc.cu); err = device error word.
-cudaError_t launch_score_tc(const float* qbar, const float* kbar, const float* vbar, int B, int Hq, int Hkv, int nb,
-                            int d, float tau, int metric, float* scores, int nb_stride, unsigned* err,
-                            cudaStream_t s);
-cudaError_t launch_score(const float* qbar, const float* kbar, const float* vbar, int B, int Hq, int Hkv, int nb,
-                         int d, float tau, int metric, float* scores, int nb_stride, cudaStream_t s);
+// tcgen05 3xTF32 GEMM (score_tc.cu) over 4-D tensor maps of qhi, qlo [d, nb, Hq, B] and khi,
+// klo [d, nb, Hkv, B] (fp32, 128-byte swizzle, box 32 x 128); err = device error word.
+cudaError_t launch_score_tc(const CUtensorMap& mqh, const CUtensorMap& mql, const CUtensorMap& mkh,
+                            const CUtensorMap& mkl, const float* vbar, int B, int Hq, int Hkv, int nb, int d,
+                            float tau, int metric, float* scores, int nb_stride, unsigned* err, cudaStream_t s);
+// fp32 FMA version (score.cu); reads qhi + qlo and khi + klo.
+cudaError_t launch_score(const float* qhi, const float* qlo, const float* khi, const float* klo, const float* vbar,
+                         int B, int Hq, int Hkv, int nb, int d, float tau, int metric, float* scores, int nb_stride,
+                         cudaStream_t s);
 
 struct SelectSeqs {
     int32_t B;

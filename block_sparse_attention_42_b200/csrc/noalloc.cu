@@ -12,7 +12,7 @@ namespace {
 
 // Fixed scratch for the pooled Q/K representations and value norms.  Every GPU that loads
 // the library holds these bytes until the process exits.
-constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 // Device address of g_noalloc_scratch on the current device.  In host code the array's name

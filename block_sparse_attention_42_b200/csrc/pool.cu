@@ -8,7 +8,9 @@
 // (blockIdx.z: 0 Q, 1 K, 2 V) over all heads: every thread owns a 16-byte column vector of
 // the [token, head*d] rows and walks a strided subset of the block's tokens, so each token
 // row is read once with fully coalesced 16-byte loads.  Sums are kept in fp64 (cheap here:
-// the kernel waits on HBM) so the pooled means carry only the final fp32 rounding.
+// the kernel waits on HBM) so the pooled means carry only the final fp32 rounding.  Each Q/K
+// mean is written as two fp32 arrays, a TF32-exact high part and the remainder, which the
+// tensor-core score GEMM consumes directly (score_tc.cu).
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 
@@ -77,10 +79,20 @@ struct Elem<2> {  // fp32
 struct PoolArgs {
     TensorArg t[3];
     int H[3];
-    float* mean_out[3];  // nullptr for V
+    float* mean_out[3];  // TF32 high part of each mean; nullptr for V
+    float* lo_out[3];    // fp32 remainder: mean = mean_out + lo_out exactly
     float* vnorm_out;
     int N, d, block, nb;
 };
+
+// Stores a pooled mean as hi + lo: hi keeps the sign, exponent and top 10 mantissa bits (exact
+// in TF32, so the tensor cores read it unchanged) and lo = m - hi is exact in fp32.  A
+// non-finite mean keeps lo = 0 so that hi + lo still gives it back.
+__device__ __forceinline__ void store_split(const PoolArgs& a, int which, int64_t o, float m) {
+    const float hi = __uint_as_float(__float_as_uint(m) & 0xFFFFE000u);
+    a.mean_out[which][o] = hi;
+    a.lo_out[which][o] = isfinite(m) ? m - hi : 0.f;
+}
 
 template <int DT>
 __global__ void __launch_bounds__(kPoolThreads, 2) pool_kernel(const PoolArgs a) {
@@ -187,8 +199,7 @@ __global__ void __launch_bounds__(kPoolThreads, 2) pool_kernel(const PoolArgs a)
                 const int64_t o = ((static_cast<int64_t>(b) * H + h) * a.nb + i) * d + c0;
                 if (!is_v) {
 #pragma unroll
-                    for (int e = 0; e < V; ++e)
-                        a.mean_out[which][o + e] = static_cast<float>(acc[e] * inv_cnt * x.scale);
+                    for (int e = 0; e < V; ++e) store_split(a, which, o + e, static_cast<float>(acc[e] * inv_cnt * x.scale));
                 } else if (c0 == 0) {
                     a.vnorm_out[(static_cast<int64_t>(b) * H + h) * a.nb + i] =
                         static_cast<float>(nacc * inv_cnt * x.scale);
@@ -208,7 +219,7 @@ __global__ void __launch_bounds__(kPoolThreads, 2) pool_kernel(const PoolArgs a)
                 if (!is_v) {
 #pragma unroll
                     for (int e = 0; e < V; ++e)
-                        a.mean_out[which][o + e] = static_cast<float>(red[threadIdx.x][e] * inv_cnt * x.scale);
+                        store_split(a, which, o + e, static_cast<float>(red[threadIdx.x][e] * inv_cnt * x.scale));
                 } else if (c0 == 0) {
                     a.vnorm_out[(static_cast<int64_t>(b) * H + h) * a.nb + i] =
                         static_cast<float>(red[threadIdx.x][V] * inv_cnt * x.scale);
@@ -221,7 +232,7 @@ __global__ void __launch_bounds__(kPoolThreads, 2) pool_kernel(const PoolArgs a)
 }  // namespace
 
 cudaError_t launch_pool(int dtype, TensorArg q, TensorArg k, TensorArg v, int B, int N, int Hq, int Hkv, int d,
-                        int block, float* qbar, float* kbar, float* vbar, cudaStream_t s) {
+                        int block, float* qbar, float* qlo, float* kbar, float* klo, float* vbar, cudaStream_t s) {
     PoolArgs a;
     a.t[0] = q;
     a.t[1] = k;
@@ -232,6 +243,9 @@ cudaError_t launch_pool(int dtype, TensorArg q, TensorArg k, TensorArg v, int B,
     a.mean_out[0] = qbar;
     a.mean_out[1] = kbar;
     a.mean_out[2] = nullptr;
+    a.lo_out[0] = qlo;
+    a.lo_out[1] = klo;
+    a.lo_out[2] = nullptr;
     a.vnorm_out = vbar;
     a.N = N;
     a.d = d;

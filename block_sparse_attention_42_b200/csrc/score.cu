@@ -21,10 +21,16 @@ namespace {
 constexpr int kTile = 64;
 constexpr int kKc = 32;
 
-__global__ void __launch_bounds__(256) score_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar,
-                                                    const float* __restrict__ vbar, int Hq, int Hkv, int nb,
-                                                    int d, float tau, int metric, float* __restrict__ S,
-                                                    int nbs) {
+__device__ __forceinline__ float4 load_mean(const float* hi, const float* lo, int64_t o) {
+    const float4 h = *reinterpret_cast<const float4*>(hi + o);
+    const float4 l = *reinterpret_cast<const float4*>(lo + o);
+    return make_float4(h.x + l.x, h.y + l.y, h.z + l.z, h.w + l.w);
+}
+
+__global__ void __launch_bounds__(256)
+    score_kernel(const float* __restrict__ qhi, const float* __restrict__ qlo, const float* __restrict__ khi,
+                 const float* __restrict__ klo, const float* __restrict__ vbar, int Hq, int Hkv, int nb, int d,
+                 float tau, int metric, float* __restrict__ S, int nbs) {
     __shared__ __align__(16) float As[kKc][kTile + 4];
     __shared__ __align__(16) float Bs[kKc][kTile + 4];
     __shared__ float lv[kTile];
@@ -39,8 +45,8 @@ __global__ void __launch_bounds__(256) score_kernel(const float* __restrict__ qb
     const int hk = h / (Hq / Hkv);
     const int i0 = ti * kTile, j0 = tj * kTile;
 
-    const float* A = qbar + (static_cast<int64_t>(b) * Hq + h) * nb * d;
-    const float* Bm = kbar + (static_cast<int64_t>(b) * Hkv + hk) * nb * d;
+    const int64_t qo = (static_cast<int64_t>(b) * Hq + h) * nb * d;
+    const int64_t ko = (static_cast<int64_t>(b) * Hkv + hk) * nb * d;
     const float* vb = vbar + (static_cast<int64_t>(b) * Hkv + hk) * nb;
 
     const int tid = threadIdx.x;
@@ -64,8 +70,9 @@ __global__ void __launch_bounds__(256) score_kernel(const float* __restrict__ qb
             const int idx = tid + rep * 256;     // 0..511
             const int row = idx / 8, q4 = (idx % 8) * 4;
             float4 av = make_float4(0.f, 0.f, 0.f, 0.f), bv = av;
-            if (i0 + row < nb) av = *reinterpret_cast<const float4*>(A + static_cast<int64_t>(i0 + row) * d + k0 + q4);
-            if (j0 + row < nb) bv = *reinterpret_cast<const float4*>(Bm + static_cast<int64_t>(j0 + row) * d + k0 + q4);
+            // The pooled means are stored as hi + lo; the fp32 sum is exact.
+            if (i0 + row < nb) av = load_mean(qhi, qlo, qo + static_cast<int64_t>(i0 + row) * d + k0 + q4);
+            if (j0 + row < nb) bv = load_mean(khi, klo, ko + static_cast<int64_t>(j0 + row) * d + k0 + q4);
             As[q4 + 0][row] = av.x;
             As[q4 + 1][row] = av.y;
             As[q4 + 2][row] = av.z;
@@ -117,11 +124,12 @@ __global__ void __launch_bounds__(256) score_kernel(const float* __restrict__ qb
 
 }  // namespace
 
-cudaError_t launch_score(const float* qbar, const float* kbar, const float* vbar, int B, int Hq, int Hkv, int nb,
-                         int d, float tau, int metric, float* scores, int nb_stride, cudaStream_t s) {
+cudaError_t launch_score(const float* qhi, const float* qlo, const float* khi, const float* klo, const float* vbar,
+                         int B, int Hq, int Hkv, int nb, int d, float tau, int metric, float* scores, int nb_stride,
+                         cudaStream_t s) {
     const int nt = (nb + kTile - 1) / kTile;
     dim3 grid(nt * (nt + 1) / 2, Hq, B);
-    score_kernel<<<grid, 256, 0, s>>>(qbar, kbar, vbar, Hq, Hkv, nb, d, tau, metric, scores, nb_stride);
+    score_kernel<<<grid, 256, 0, s>>>(qhi, qlo, khi, klo, vbar, Hq, Hkv, nb, d, tau, metric, scores, nb_stride);
     return cudaGetLastError();
 }
 

@@ -9,19 +9,26 @@
 //                                                   * vbar for OAM_MUL), j <= i; -inf above.
 //
 // The scores decide integer top-k lists, so the product must be fp32-accurate; TF32 or BF16
-// alone would move scores by ~1e-3 and reorder near-equal candidates.  Each fp32 operand is
-// split into hi = x with its 13 low mantissa bits cleared (exactly representable in TF32) and
-// lo = x - hi (exact in fp32), and the tensor cores accumulate hi*hi + hi*lo + lo*hi in fp32
-// (kind::tf32).  The dropped lo*lo term and the TF32 truncation of lo are ~2^-20 of the
-// product.
+// alone would move scores by ~1e-3 and reorder near-equal candidates.  The pooling kernel
+// stores each pooled fp32 value x split as hi = x with its 13 low mantissa bits cleared (exact
+// in TF32) and lo = x - hi (exact in fp32), and the tensor cores accumulate hi*hi + hi*lo +
+// lo*hi in fp32 (kind::tf32).  The dropped lo*lo term and the TF32 truncation of lo are ~2^-20
+// of the product.
 //
-// One CTA (128 threads) computes one 128 x 128 tile (query blocks x key blocks) of one query
-// head; tiles wholly above the diagonal are not launched.  The contraction runs over head_dim
-// in chunks of 32 values (one 128-byte swizzled row): all threads load the fp32 chunk of Qbar
-// and Kbar, split it and store hi / lo into shared memory in the 128-byte-swizzled K-major
-// layout; thread 0 issues the 3 x 4 MMAs of the chunk into TMEM and commits them to an
-// mbarrier that gates the next chunk.  The epilogue reads the accumulator row of each thread
-// from TMEM and writes the scores.  Every wait is bounded.
+// A persistent GEMM over the causal 128 x 128 tiles (query blocks x key blocks) of every
+// query head, one CTA per SM (6 warps):
+//   warp 0      TMA producer: per 32-value chunk of head_dim, the hi / lo rows of the tile's
+//               Qbar and Kbar (4 x 16 KB, 128-byte swizzle, rows past nb read as zeros) into a
+//               ring of 3 stages
+//   warp 1      MMA issuer (TMEM owner): 3 x 4 MMAs per chunk into one of two TMEM
+//               accumulators (128 columns each), so the next tile runs while the last drains
+//   warps 2-9   epilogue, two warps per TMEM lane quarter, each with half of the columns:
+//               ln vbar of the tile's 128 key blocks once into shared memory (one per thread
+//               of the first half), then per 32 columns tcgen05.ld of the thread's row,
+//               tau * acc (+ ln vbar), -inf above the diagonal, and a transpose through a
+//               per-warp shared buffer so that each store instruction writes whole 128-byte
+//               score-row segments
+// Every wait is bounded (sm100.cuh).
 #include <cmath>
 
 #include "internal.h"
@@ -30,179 +37,303 @@
 namespace bsa {
 namespace {
 
-constexpr int kTileS = 128;       // query blocks x key blocks per CTA
-constexpr int kChunk = 32;        // fp32 values of head_dim per chunk (one 128-byte row)
-constexpr int kOpBytes = kTileS * 128;  // one operand chunk in shared memory (16 KB)
+constexpr int kTileS = 128;
+constexpr int kChunk = 32;              // fp32 values of head_dim per chunk (one 128-byte row)
+constexpr int kOpBytes = kTileS * 128;  // one operand chunk (16 KB)
+constexpr int kStageBytes = 4 * kOpBytes;
+constexpr int kStagesS = 3;
+constexpr int kThreadsS = 320;
 
-struct ScoreSmem {
-    uint8_t a_hi[kOpBytes], a_lo[kOpBytes], b_hi[kOpBytes], b_lo[kOpBytes];
-    float lv[kTileS];
-    uint64_t mma_done;
+struct ScoreBars {
+    uint64_t full[kStagesS], empty[kStagesS];
+    uint64_t acc_full[2], acc_empty[2];
+    uint64_t drain, tmem_free;
     uint32_t tmem_slot;
     int abort_flag;
 };
+constexpr int kEpiWarps = 8;
+constexpr int kEpiThreads = kEpiWarps * 32;
+static_assert(kThreadsS == 64 + kEpiThreads, "producer + MMA warps + epilogue");
+constexpr int kTrBytes = kEpiWarps * 32 * 32 * 4;  // epilogue transpose buffers, 32 x 32 fp32 per warp
+constexpr int kLvBytes = 2 * kTileS * 4;    // per-column terms of the last two tiles
+constexpr int kScoreSmem = kStagesS * kStageBytes + kTrBytes + kLvBytes + 256 + 1024;  // + barriers, slack
+static_assert(kScoreSmem <= 227 * 1024, "shared memory per CTA");
 
-__device__ __forceinline__ float tf32_hi(float x) { return __uint_as_float(__float_as_uint(x) & 0xFFFFE000u); }
-
-// 128 rows x 32 fp32 of `src` (row stride d floats, rows >= n_valid read as zero) -> hi / lo
-// operands in the 128-byte-swizzled K-major layout.
-__device__ __forceinline__ void stage_chunk(const float* __restrict__ src, int row0, int n_valid, int d, int k0,
-                                            uint8_t* hi, uint8_t* lo) {
-#pragma unroll
-    for (int rep = 0; rep < kTileS * 8 / 128; ++rep) {
-        const int idx = threadIdx.x + rep * 128;  // 0 .. 1023
-        const int r = idx / 8, c = idx % 8;        // row, 16-byte chunk within the 128-byte row
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (row0 + r < n_valid) v = __ldg(reinterpret_cast<const float4*>(src + static_cast<int64_t>(row0 + r) * d + k0) + c);
-        const float4 vh = make_float4(tf32_hi(v.x), tf32_hi(v.y), tf32_hi(v.z), tf32_hi(v.w));
-        const float4 vl = make_float4(v.x - vh.x, v.y - vh.y, v.z - vh.z, v.w - vh.w);
-        const int off = r * 128 + ((c ^ (r & 7)) * 16);
-        *reinterpret_cast<float4*>(hi + off) = vh;
-        *reinterpret_cast<float4*>(lo + off) = vl;
-    }
+// Barrier 1 over the epilogue warps, returning whether `p` held in every thread.
+__device__ __forceinline__ bool epilogue_all(bool p) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred pi, po;\n\t"
+        "setp.ne.u32 pi, %1, 0;\n\t"
+        "bar.red.and.pred po, 1, 256, pi;\n\t"
+        "selp.u32 %0, 1, 0, po;\n\t}\n"
+        : "=r"(r)
+        : "r"(static_cast<uint32_t>(p))
+        : "memory");
+    return r != 0;
 }
 
-template <int D>
-__global__ void __launch_bounds__(128) score_tf32x3_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar,
-                                                           const float* __restrict__ vbar, int Hq, int Hkv, int nb,
-                                                           float tau, int metric, float* __restrict__ S, int nbs,
-                                                           unsigned* err) {
-    extern __shared__ uint8_t smem_raw[];
-    ScoreSmem& sm = *reinterpret_cast<ScoreSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const int tid = threadIdx.x, warp = tid / 32;
+struct TileRC {
+    int b, h, hk, i0, j0;
+};
 
-    // Lower-triangular tile pair (ti, tj), tj <= ti.
-    const int x = blockIdx.x;
+// Tile t -> (sequence, head, first query block, first key block); per head the causal tile
+// pairs (ti, tj), tj <= ti, in row-major order.
+__device__ __forceinline__ TileRC decode_score_tile(int t, int nt, int Hq, int G) {
+    const int per = nt * (nt + 1) / 2;
+    const int bh = t / per;
+    const int x = t % per;
     int ti = static_cast<int>((sqrtf(8.f * x + 1.f) - 1.f) * 0.5f);
     while ((ti + 1) * (ti + 2) / 2 <= x) ++ti;
     while (ti * (ti + 1) / 2 > x) --ti;
     const int tj = x - ti * (ti + 1) / 2;
-    const int h = blockIdx.y, b = blockIdx.z;
-    const int hk = h / (Hq / Hkv);
-    const int i0 = ti * kTileS, j0 = tj * kTileS;
-    const float* A = qbar + (static_cast<int64_t>(b) * Hq + h) * nb * D;
-    const float* Bm = kbar + (static_cast<int64_t>(b) * Hkv + hk) * nb * D;
-    const float* vb = vbar + (static_cast<int64_t>(b) * Hkv + hk) * nb;
+    TileRC r;
+    r.h = bh % Hq;
+    r.b = bh / Hq;
+    r.hk = r.h / G;
+    r.i0 = ti * kTileS;
+    r.j0 = tj * kTileS;
+    return r;
+}
 
-    if (tid == 0) {
-        mbar_init(&sm.mma_done, 1);
-        sm.abort_flag = 0;
+template <int D>
+__global__ void __launch_bounds__(kThreadsS, 1)
+    score_tf32x3_kernel(const __grid_constant__ CUtensorMap mqh, const __grid_constant__ CUtensorMap mql,
+                        const __grid_constant__ CUtensorMap mkh, const __grid_constant__ CUtensorMap mkl,
+                        const float* __restrict__ vbar, int Hq, int Hkv, int nb, float tau, int metric,
+                        float* __restrict__ S, int nbs, int total_tiles, unsigned* err) {
+    constexpr int NCH = D / kChunk;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    float* tr_all = reinterpret_cast<float*>(smem + kStagesS * kStageBytes);
+    float* lv_all = reinterpret_cast<float*>(smem + kStagesS * kStageBytes + kTrBytes);
+    ScoreBars* bars = reinterpret_cast<ScoreBars*>(smem + kStagesS * kStageBytes + kTrBytes + kLvBytes);
+    volatile int* abort_flag = &bars->abort_flag;
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int nt = (nb + kTileS - 1) / kTileS;
+    const int G = Hq / Hkv;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStagesS; ++s) {
+            mbar_init(&bars->full[s], 1);
+            mbar_init(&bars->empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&bars->acc_full[a], 1);
+            mbar_init(&bars->acc_empty[a], kEpiThreads);
+        }
+        mbar_init(&bars->drain, 1);
+        mbar_init(&bars->tmem_free, kEpiThreads);
+        bars->abort_flag = 0;
         fence_barrier_init();
+        tma_prefetch_desc(&mqh);
+        tma_prefetch_desc(&mql);
+        tma_prefetch_desc(&mkh);
+        tma_prefetch_desc(&mkl);
     }
-    {
-        const int j = j0 + tid;
-        const float a = j < nb ? vb[j] : 1.f;
-        sm.lv[tid] = metric == 0 ? logf(a) : a;
-    }
-    if (warp == 0) {
-        tmem_alloc(&sm.tmem_slot, kTileS);
+    __syncwarp();
+    if (warp == 1) {
+        tmem_alloc(&bars->tmem_slot, 2 * kTileS);
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = sm.tmem_slot;
-    const uint32_t idesc = make_idesc(kTileS, kTileS, 2u /* TF32 */, false, false);
+    const uint32_t tmem = bars->tmem_slot;
 
-    bool ok = true;
-    constexpr int NCH = D / kChunk;
-#pragma unroll 1
-    for (int ch = 0; ch < NCH; ++ch) {
-        if (ch > 0) {
-            // The previous chunk's MMAs have read the shared-memory operands.
-            ok = mbar_wait(&sm.mma_done, (ch - 1) & 1, &sm.abort_flag, err);
-            if (__syncthreads_or(!ok)) break;
-            tc_fence_after();
-        }
-        stage_chunk(A, i0, nb, D, ch * kChunk, sm.a_hi, sm.a_lo);
-        stage_chunk(Bm, j0, nb, D, ch * kChunk, sm.b_hi, sm.b_lo);
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t ah = smem_u32(sm.a_hi), al = smem_u32(sm.a_lo);
-            const uint32_t bh = smem_u32(sm.b_hi), bl = smem_u32(sm.b_lo);
-#pragma unroll
-            for (int kk = 0; kk < kChunk / 8; ++kk) {  // 8 tf32 = 32 bytes of K per MMA
-                const uint32_t o = kk * 32;
-                const uint32_t first = (ch == 0 && kk == 0) ? 0u : 1u;
-                mma_tf32_ss(tmem, smem_desc_sw128(ah + o, 16, 1024), smem_desc_sw128(bh + o, 16, 1024), idesc, first);
-                mma_tf32_ss(tmem, smem_desc_sw128(ah + o, 16, 1024), smem_desc_sw128(bl + o, 16, 1024), idesc, 1u);
-                mma_tf32_ss(tmem, smem_desc_sw128(al + o, 16, 1024), smem_desc_sw128(bh + o, 16, 1024), idesc, 1u);
-            }
-            tc_commit(&sm.mma_done);
-        }
-        __syncwarp();
-    }
-    if (ok) {
-        ok = mbar_wait(&sm.mma_done, (NCH - 1) & 1, &sm.abort_flag, err);
-        ok = !__syncthreads_or(!ok);
-    }
-    if (ok) {
-        tc_fence_after();
-        // Epilogue: thread t owns accumulator row t (TMEM lane t).
-        const int i = i0 + tid;
-        const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-        float* out = S + (static_cast<int64_t>(b) * Hq + h) * nbs * nbs + static_cast<int64_t>(i) * nbs;
-#pragma unroll
-        for (int c0 = 0; c0 < kTileS; c0 += 32) {
-            uint32_t r[32];
-            tmem_ld32(trow + c0, r);
-            if (i < nb) {
-#pragma unroll
-                for (int q = 0; q < 32; q += 4) {
-                    float v4[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int jj = c0 + q + e, j = j0 + jj;
-                        float sc = tau * __uint_as_float(r[q + e]);
-                        if (metric == 0)
-                            sc += sm.lv[jj];
-                        else if (metric == 2)
-                            sc *= sm.lv[jj];
-                        v4[e] = j > i ? -INFINITY : sc;
-                    }
-                    const int j = j0 + c0 + q;
-                    // A 16-byte store only where the row stride leaves out + j 16-byte aligned.
-                    if (j + 3 < nb && (reinterpret_cast<uintptr_t>(out + j) & 15u) == 0) {
-                        *reinterpret_cast<float4*>(out + j) = make_float4(v4[0], v4[1], v4[2], v4[3]);
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            if (j + e < nb) out[j + e] = v4[e];
-                    }
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            uint32_t ring = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; ok && t < total_tiles; t += gridDim.x) {
+                const TileRC r = decode_score_tile(t, nt, Hq, G);
+                for (int c = 0; ok && c < NCH; ++c) {
+                    const int st = ring % kStagesS;
+                    ok = mbar_wait(&bars->empty[st], ((ring / kStagesS) & 1) ^ 1, abort_flag, err);
+                    if (!ok) break;
+                    uint8_t* dst = smem + st * kStageBytes;
+                    uint64_t* fb = &bars->full[st];
+                    mbar_arrive_expect_tx(fb, kStageBytes);
+                    tma_load_4d(dst, &mqh, fb, c * kChunk, r.i0, r.h, r.b);
+                    tma_load_4d(dst + kOpBytes, &mql, fb, c * kChunk, r.i0, r.h, r.b);
+                    tma_load_4d(dst + 2 * kOpBytes, &mkh, fb, c * kChunk, r.j0, r.hk, r.b);
+                    tma_load_4d(dst + 3 * kOpBytes, &mkl, fb, c * kChunk, r.j0, r.hk, r.b);
+                    ++ring;
                 }
             }
+            // Every issued copy must land before the shared memory goes away.
+            volatile int no_abort = 0;
+            for (uint32_t q = ring > kStagesS ? ring - kStagesS : 0; q < ring; ++q)
+                mbar_wait(&bars->full[q % kStagesS], (q / kStagesS) & 1, &no_abort, err);
         }
-    } else if (tid == 0) {
-        // Drain the MMAs in flight before the shared memory and TMEM go away.
-        volatile int no_abort = 0;
-        tc_commit(&sm.mma_done);
-        mbar_wait(&sm.mma_done, NCH & 1, &no_abort, err);
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc = make_idesc(kTileS, kTileS, 2u /* TF32 */, false, false);
+            uint32_t ring = 0, tc = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; ok && t < total_tiles; t += gridDim.x, ++tc) {
+                const uint32_t ab = tc & 1;
+                if (tc >= 2) {
+                    // The epilogue has drained this accumulator's previous tile.
+                    ok = mbar_wait(&bars->acc_empty[ab], ((tc / 2) - 1) & 1, abort_flag, err);
+                    if (!ok) break;
+                    tc_fence_after();
+                }
+                const uint32_t acc = tmem + ab * kTileS;
+                for (int c = 0; ok && c < NCH; ++c) {
+                    const int st = ring % kStagesS;
+                    ok = mbar_wait(&bars->full[st], (ring / kStagesS) & 1, abort_flag, err);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t ah = smem_u32(smem + st * kStageBytes);
+                    const uint32_t al = ah + kOpBytes, bh = ah + 2 * kOpBytes, bl = ah + 3 * kOpBytes;
+#pragma unroll
+                    for (int kk = 0; kk < kChunk / 8; ++kk) {  // 8 tf32 = 32 bytes of K per MMA
+                        const uint32_t o = kk * 32;
+                        const uint32_t first = (c == 0 && kk == 0) ? 0u : 1u;
+                        mma_tf32_ss(acc, smem_desc_sw128(ah + o, 16, 1024), smem_desc_sw128(bh + o, 16, 1024), idesc,
+                                    first);
+                        mma_tf32_ss(acc, smem_desc_sw128(ah + o, 16, 1024), smem_desc_sw128(bl + o, 16, 1024), idesc, 1u);
+                        mma_tf32_ss(acc, smem_desc_sw128(al + o, 16, 1024), smem_desc_sw128(bh + o, 16, 1024), idesc, 1u);
+                    }
+                    tc_commit(&bars->empty[st]);
+                    ++ring;
+                }
+                if (ok) tc_commit(&bars->acc_full[ab]);
+            }
+            tc_commit(&bars->drain);
+            volatile int no_abort = 0;
+            mbar_wait(&bars->drain, 0, &no_abort, err);
+            mbar_wait(&bars->tmem_free, 0, &no_abort, err);
+        }
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, 2 * kTileS);
+        return;
+    } else {
+        // ------------------------------------------------------------ epilogue (warps 2-9)
+        const int ew = warp - 2;
+        const int quad = warp % 4;          // TMEM lanes 32 * quad .. 32 * quad + 31
+        const int half = ew / 4;            // columns 64 * half .. 64 * half + 63
+        const int row = quad * 32 + lane;
+        const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+        float* tr = tr_all + ew * 32 * 32;
+        // 16-byte stores need every score row segment 16-byte aligned.
+        const bool vec_ok = (nbs % 4) == 0 && (reinterpret_cast<uintptr_t>(S) & 15u) == 0;
+        uint32_t tc = 0;
+        for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++tc) {
+            const uint32_t ab = tc & 1;
+            const TileRC r = decode_score_tile(t, nt, Hq, G);
+            // This tile's per-column term: ln vbar (OAM), vbar (OAM_MUL); one column per thread
+            // of the first half.  lv_all holds two tiles' terms, so the write below cannot race
+            // the reads of the previous tile: every epilogue thread has passed that tile's
+            // barrier, which comes after its reads of the tile before.
+            float* lv = lv_all + ab * kTileS;
+            if (half == 0) {
+                const int j = r.j0 + row;
+                float a = 0.f;
+                if (metric != 1 && j < nb) {
+                    a = __ldg(vbar + (static_cast<int64_t>(r.b) * Hkv + r.hk) * nb + j);
+                    if (metric == 0) a = logf(a);
+                }
+                lv[row] = a;
+            }
+            // One barrier per tile for all epilogue threads, also on the way out: a thread whose
+            // wait gave up makes every epilogue thread leave at the same tile.
+            const bool ok = mbar_wait(&bars->acc_full[ab], (tc / 2) & 1, abort_flag, err);
+            if (!epilogue_all(ok)) break;
+            tc_fence_after();
+            const bool diag = r.i0 == r.j0;  // the only tiles with entries above the diagonal
+            float* out_head = S + (static_cast<int64_t>(r.b) * Hq + r.h) * nbs * nbs;
+#pragma unroll 1
+            for (int g = 0; g < 2; ++g) {
+                const int c0 = half * 64 + g * 32;
+                uint32_t v[32];
+                tmem_ld32(tmem + lane_base + ab * kTileS + c0, v);
+                if (g == 1) {
+                    // The accumulator is in registers: the MMA warp may reuse it.
+                    tc_fence_before();
+                    mbar_arrive(&bars->acc_empty[ab]);
+                }
+                // Row `lane` of this warp's 32 x 32 buffer, 16-byte chunks rotated by the row
+                // (chunk q at q ^ (row & 7)) so that both the row writes here and the column
+                // reads below are free of bank conflicts.
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const float4 l4 = *reinterpret_cast<const float4*>(lv + c0 + q * 4);
+                    const float la[4] = {l4.x, l4.y, l4.z, l4.w};
+                    float o[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float acc = __uint_as_float(v[q * 4 + e]);
+                        float sc;
+                        if (metric == 0)
+                            sc = fmaf(tau, acc, la[e]);
+                        else if (metric == 2)
+                            sc = tau * acc * la[e];
+                        else
+                            sc = tau * acc;
+                        if (diag && c0 + q * 4 + e > row) sc = -INFINITY;
+                        o[e] = sc;
+                    }
+                    *reinterpret_cast<float4*>(tr + lane * 32 + ((q ^ (lane & 7)) * 4)) =
+                        make_float4(o[0], o[1], o[2], o[3]);
+                }
+                __syncwarp();
+                // 8 lanes per score row, 4 rows per instruction.
+#pragma unroll
+                for (int p = 0; p < 8; ++p) {
+                    const int rr = p * 4 + lane / 8, cq = lane % 8;
+                    const float4 o = *reinterpret_cast<const float4*>(tr + rr * 32 + ((cq ^ (rr & 7)) * 4));
+                    const int gi = r.i0 + quad * 32 + rr, gj = r.j0 + c0 + cq * 4;
+                    if (gi < nb) {
+                        float* dst = out_head + static_cast<int64_t>(gi) * nbs + gj;
+                        if (vec_ok && gj + 3 < nb) {
+                            *reinterpret_cast<float4*>(dst) = o;
+                        } else {
+                            const float oe[4] = {o.x, o.y, o.z, o.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e)
+                                if (gj + e < nb) dst[e] = oe[e];
+                        }
+                    }
+                }
+                __syncwarp();
+            }
+        }
+        tc_fence_before();
+        mbar_arrive(&bars->tmem_free);
+        return;
     }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    if (warp == 0) tmem_dealloc(tmem, kTileS);
 }
 
 }  // namespace
 
-cudaError_t launch_score_tc(const float* qbar, const float* kbar, const float* vbar, int B, int Hq, int Hkv, int nb,
-                            int d, float tau, int metric, float* scores, int nb_stride, unsigned* err,
-                            cudaStream_t s) {
+cudaError_t launch_score_tc(const CUtensorMap& mqh, const CUtensorMap& mql, const CUtensorMap& mkh,
+                            const CUtensorMap& mkl, const float* vbar, int B, int Hq, int Hkv, int nb, int d,
+                            float tau, int metric, float* scores, int nb_stride, unsigned* err, cudaStream_t s) {
     const int nt = (nb + kTileS - 1) / kTileS;
-    dim3 grid(nt * (nt + 1) / 2, Hq, B);
-    const int smem = static_cast<int>(sizeof(ScoreSmem)) + 1024;
+    const long long total = static_cast<long long>(nt) * (nt + 1) / 2 * Hq * B;
+    if (total > 0x7FFFFFFFll) return cudaErrorInvalidValue;  // tile indices are int
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const unsigned grid = static_cast<unsigned>(total < sms ? total : sms);
     if (d == 128) {
-        cudaError_t e = cudaFuncSetAttribute(score_tf32x3_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        cudaError_t e = cudaFuncSetAttribute(score_tf32x3_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             kScoreSmem);
         if (e != cudaSuccess) return e;
-        score_tf32x3_kernel<128><<<grid, 128, smem, s>>>(qbar, kbar, vbar, Hq, Hkv, nb, tau, metric, scores, nb_stride, err);
+        score_tf32x3_kernel<128><<<grid, kThreadsS, kScoreSmem, s>>>(mqh, mql, mkh, mkl, vbar, Hq, Hkv, nb, tau, metric,
+                                                                      scores, nb_stride, static_cast<int>(total), err);
     } else if (d == 64) {
-        cudaError_t e = cudaFuncSetAttribute(score_tf32x3_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        cudaError_t e = cudaFuncSetAttribute(score_tf32x3_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             kScoreSmem);
         if (e != cudaSuccess) return e;
-        score_tf32x3_kernel<64><<<grid, 128, smem, s>>>(qbar, kbar, vbar, Hq, Hkv, nb, tau, metric, scores, nb_stride, err);
+        score_tf32x3_kernel<64><<<grid, kThreadsS, kScoreSmem, s>>>(mqh, mql, mkh, mkl, vbar, Hq, Hkv, nb, tau, metric,
+                                                                     scores, nb_stride, static_cast<int>(total), err);
     } else {
         return cudaErrorInvalidValue;
     }

@@ -89,7 +89,8 @@ size_t bsa_score_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int32_t nb,
  * that touch the diagonal are -inf, tiles wholly above it are not written.  The product runs
  * on the tensor cores as three TF32 products (hi*hi + hi*lo + lo*hi of each operand's split),
  * fp32-accurate.  ws: device workspace of at least bsa_score_workspace_bytes() bytes, 256-byte
- * aligned. */
+ * aligned; it receives the pooled means (each split into that TF32 high part and its fp32
+ * remainder) and the value norms. */
 bsa_status_t stem_score(bsa_tensor_t q, bsa_tensor_t k, bsa_tensor_t v, int32_t B, int32_t N,
                         int32_t Hq, int32_t Hkv, int32_t d, int32_t block, int32_t metric,
                         float softmax_scale, float* scores, int32_t nb_stride, void* ws,
@@ -143,8 +144,8 @@ bsa_status_t bsa_prefill_paged(bsa_tensor_t q, bsa_tensor_t out, const int32_t* 
  *
  * Arguments, layouts, results and errors are those of stem_score.  The pooled Q/K
  * representations and value norms that stem_score keeps in `ws` live instead in a fixed
- * 16 MiB array inside the library, which every GPU that loads the library holds until the
- * process exits.  Problems that need more than that (bsa_score_workspace_bytes() > 16 MiB,
+ * 32 MiB array inside the library, which every GPU that loads the library holds until the
+ * process exits.  Problems that need more than that (bsa_score_workspace_bytes() > 32 MiB,
  * e.g. beyond about 58K tokens at 64 query / 8 KV heads, d = 128, block 128) are rejected
  * with BSA_ERR_UNSUPPORTED and a message naming both sizes; nothing is launched.  The call
  * itself allocates nothing: no cudaMalloc, cudaFree or allocating library routine.

@@ -2,7 +2,7 @@
 
 Some callers cannot allocate device memory (a plain C program that links only this
 library, or a runtime whose memory pool owns all of HBM); this entry point keeps the pooled
-block representations in a fixed 16 MiB array inside the library instead of a caller
+block representations in a fixed 32 MiB array inside the library instead of a caller
 workspace.  These tests call it through the C ABI and check it against stem_score on two
 calls in a row (different inputs, so stale scratch contents would show up), and that a
 problem too large for the fixed scratch is refused with a clear error.
