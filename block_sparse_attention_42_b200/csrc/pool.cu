@@ -8,7 +8,9 @@
 // (blockIdx.z: 0 Q, 1 K, 2 V) over all heads: every thread owns a 16-byte column vector of
 // the [token, head*d] rows and walks a strided subset of the block's tokens, so each token
 // row is read once with fully coalesced 16-byte loads.  Sums are kept in fp64 (cheap here:
-// the kernel waits on HBM) so the pooled means carry only the final fp32 rounding.  Each Q/K
+// the kernel waits on HBM) so the pooled means carry only the final fp32 rounding.  What
+// bounds it is the number of 16-byte loads in flight per SM, so the E4M3 instantiation keeps
+// its fp64 sums in shared memory and its registers at 64 per thread, for four CTAs per SM.  Each Q/K
 // mean is written as two fp32 arrays, a TF32-exact high part and the remainder, which the
 // tensor-core score GEMM consumes directly (score_tc.cu).
 #include <cuda_bf16.h>
@@ -65,6 +67,41 @@ struct Elem<1> {  // e4m3
         }
     }
 };
+// Four E4M3 codes of w -> two f16x2 words holding each code's value times 2^-8, exactly (an
+// E4M3 code read as f16 with its 7 exponent/mantissa bits moved to f16 bits 13..7: the
+// exponent bias goes from 7 to 15, subnormals map to subnormals).  h01 holds codes 0 (low
+// half) and 1, h23 codes 2 and 3.  The NaN codes come out finite (+-480 * 2^-8); callers test
+// for them separately.
+__device__ __forceinline__ void e4m3x4_to_f16x2(uint32_t w, uint32_t& h01, uint32_t& h23) {
+    const uint32_t x01 = __byte_perm(w, 0u, 0x1404);  // code 1 << 24 | code 0 << 8
+    const uint32_t x23 = __byte_perm(w, 0u, 0x3424);  // code 3 << 24 | code 2 << 8
+    h01 = (x01 & 0x80008000u) | ((x01 >> 1) & 0x3F803F80u);
+    h23 = (x23 & 0x80008000u) | ((x23 >> 1) & 0x3F803F80u);
+}
+
+// c + the low / high f16 half of h2, rounded once to fp32 (sm_100 mixed-precision add).
+__device__ __forceinline__ float add_f16lo(uint32_t h2, float c) {
+    float d;
+    asm("{\n\t.reg .f16 l, h;\n\tmov.b32 {l, h}, %1;\n\tadd.rn.f32.f16 %0, l, %2;\n\t}" : "=f"(d) : "r"(h2), "f"(c));
+    return d;
+}
+__device__ __forceinline__ float add_f16hi(uint32_t h2, float c) {
+    float d;
+    asm("{\n\t.reg .f16 l, h;\n\tmov.b32 {l, h}, %1;\n\tadd.rn.f32.f16 %0, h, %2;\n\t}" : "=f"(d) : "r"(h2), "f"(c));
+    return d;
+}
+// c + half * half (low / high half of h2), one fp32 rounding.
+__device__ __forceinline__ float sq_f16lo(uint32_t h2, float c) {
+    float d;
+    asm("{\n\t.reg .f16 l, h;\n\tmov.b32 {l, h}, %1;\n\tfma.rn.f32.f16 %0, l, l, %2;\n\t}" : "=f"(d) : "r"(h2), "f"(c));
+    return d;
+}
+__device__ __forceinline__ float sq_f16hi(uint32_t h2, float c) {
+    float d;
+    asm("{\n\t.reg .f16 l, h;\n\tmov.b32 {l, h}, %1;\n\tfma.rn.f32.f16 %0, h, h, %2;\n\t}" : "=f"(d) : "r"(h2), "f"(c));
+    return d;
+}
+
 template <>
 struct Elem<2> {  // fp32
     static constexpr int kVec = 4;
@@ -95,7 +132,7 @@ __device__ __forceinline__ void store_split(const PoolArgs& a, int which, int64_
 }
 
 template <int DT>
-__global__ void __launch_bounds__(kPoolThreads, 2) pool_kernel(const PoolArgs a) {
+__global__ void __launch_bounds__(kPoolThreads, DT == 1 ? 4 : 2) pool_kernel(const PoolArgs a) {
     constexpr int V = Elem<DT>::kVec;
     const int which = blockIdx.z;
     const TensorArg x = a.t[which];
@@ -108,6 +145,9 @@ __global__ void __launch_bounds__(kPoolThreads, 2) pool_kernel(const PoolArgs a)
     const int t_lo = i * a.block;
     const int t_hi = min(a.N, t_lo + a.block);
     const double inv_cnt = 1.0 / static_cast<double>(t_hi - t_lo);
+    // E4M3 sums are of the values times 2^-8 (below); the final scale puts the 2^8 back, with
+    // the same roundings as unscaled sums would get.
+    const double scale = static_cast<double>(x.scale) * (DT == 1 ? 256.0 : 1.0);
     const bool is_v = (which == 2);
 
     __shared__ double red[kPoolThreads][V + 1];
@@ -120,12 +160,21 @@ __global__ void __launch_bounds__(kPoolThreads, 2) pool_kernel(const PoolArgs a)
         const bool live = active_tg && v < vpt;
         const int h = live ? v / vec_per_head : 0;
         const int c0 = live ? (v % vec_per_head) * V : 0;
-        double acc[V];
+        // fp64 sums: in registers for BF16 / fp32; for E4M3, in this thread's row of `red`
+        // (read and written only by this thread until the reduction below), which leaves the
+        // registers to keep more loads in flight.
+        double acc[DT == 1 ? 1 : V];
 #pragma unroll
-        for (int e = 0; e < V; ++e) acc[e] = 0.0;
+        for (int e = 0; e < V; ++e) {
+            if constexpr (DT == 1)
+                red[threadIdx.x][e] = 0.0;
+            else
+                acc[e] = 0.0;
+        }
         double nacc = 0.0;
         // E4M3: values are multiples of 2^-9 below 2^9, so any sum of up to 64 of them is exact
-        // in fp32; such partial sums are flushed into the fp64 sums every kFlush batches.
+        // in fp32 (also after scaling by 2^-8); such partial sums are flushed into the fp64
+        // sums every kFlush batches.
         float facc[V];
 #pragma unroll
         for (int e = 0; e < V; ++e) facc[e] = 0.f;
@@ -152,24 +201,46 @@ __global__ void __launch_bounds__(kPoolThreads, 2) pool_kernel(const PoolArgs a)
             }
 #pragma unroll
             for (int u = 0; u < kBatch; ++u) {
-                float f[V];
-                Elem<DT>::decode(raw[u], f);  // zero bits decode to +0 in every format
                 if constexpr (DT == 1) {
+                    // Sums of the codes' values times 2^-8 (f16 halves added into fp32: exact, as
+                    // above, since the scaling is a power of two); the 2^8 goes into the final
+                    // scale.  A vector holding a NaN code takes the float decode, which gives NaN.
+                    const uint32_t w[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
+                    uint32_t nan_any = 0;
 #pragma unroll
-                    for (int e = 0; e < V; ++e) facc[e] += f[e];
-                } else {
+                    for (int q = 0; q < 4; ++q) nan_any |= ((w[q] & 0x7F7F7F7Fu) + 0x01010101u) & 0x80808080u;
+                    float ss = 0.f;  // V: fp32 sum of squares, times 2^-16 (relative error ~1e-7)
+                    if (nan_any == 0) {
 #pragma unroll
-                    for (int e = 0; e < V; ++e) acc[e] += static_cast<double>(f[e]);
-                }
-                if (is_v) {
-                    if constexpr (DT == 1) {
-                        // fp32 sum of squares (relative error ~1e-7 in the norm).
-                        float ss = 0.f;
+                        for (int q = 0; q < 4; ++q) {
+                            uint32_t h01, h23;
+                            e4m3x4_to_f16x2(w[q], h01, h23);
+                            facc[4 * q + 0] = add_f16lo(h01, facc[4 * q + 0]);
+                            facc[4 * q + 1] = add_f16hi(h01, facc[4 * q + 1]);
+                            facc[4 * q + 2] = add_f16lo(h23, facc[4 * q + 2]);
+                            facc[4 * q + 3] = add_f16hi(h23, facc[4 * q + 3]);
+                            if (is_v) ss = sq_f16hi(h23, sq_f16lo(h23, sq_f16hi(h01, sq_f16lo(h01, ss))));
+                        }
+                    } else {
+                        float f[V];
+                        Elem<1>::decode(raw[u], f);
 #pragma unroll
-                        for (int e = 0; e < V; ++e) ss = fmaf(f[e], f[e], ss);
+                        for (int e = 0; e < V; ++e) {
+                            const float fs = f[e] * 0x1p-8f;
+                            facc[e] += fs;
+                            ss = fmaf(fs, fs, ss);
+                        }
+                    }
+                    if (is_v) {
                         for (int o = 1; o < vec_per_head; o <<= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
                         if (okb[u]) nacc += static_cast<double>(sqrtf(ss));
-                    } else {
+                    }
+                } else {
+                    float f[V];
+                    Elem<DT>::decode(raw[u], f);  // zero bits decode to +0 in every format
+#pragma unroll
+                    for (int e = 0; e < V; ++e) acc[e] += static_cast<double>(f[e]);
+                    if (is_v) {
                         double ss = 0.0;
 #pragma unroll
                         for (int e = 0; e < V; ++e) ss += static_cast<double>(f[e]) * static_cast<double>(f[e]);
@@ -183,7 +254,7 @@ __global__ void __launch_bounds__(kPoolThreads, 2) pool_kernel(const PoolArgs a)
                 if (++nbatch == kFlush) {
 #pragma unroll
                     for (int e = 0; e < V; ++e) {
-                        acc[e] += static_cast<double>(facc[e]);
+                        red[threadIdx.x][e] += static_cast<double>(facc[e]);
                         facc[e] = 0.f;
                     }
                     nbatch = 0;
@@ -192,22 +263,30 @@ __global__ void __launch_bounds__(kPoolThreads, 2) pool_kernel(const PoolArgs a)
         }
         if constexpr (DT == 1) {
 #pragma unroll
-            for (int e = 0; e < V; ++e) acc[e] += static_cast<double>(facc[e]);
+            for (int e = 0; e < V; ++e) red[threadIdx.x][e] += static_cast<double>(facc[e]);
         }
+        auto sum_at = [&](int e) -> double {
+            if constexpr (DT == 1)
+                return red[threadIdx.x][e];
+            else
+                return acc[e];
+        };
         if (vpt >= kPoolThreads) {
             if (live) {
                 const int64_t o = ((static_cast<int64_t>(b) * H + h) * a.nb + i) * d + c0;
                 if (!is_v) {
 #pragma unroll
-                    for (int e = 0; e < V; ++e) store_split(a, which, o + e, static_cast<float>(acc[e] * inv_cnt * x.scale));
+                    for (int e = 0; e < V; ++e) store_split(a, which, o + e, static_cast<float>(sum_at(e) * inv_cnt * scale));
                 } else if (c0 == 0) {
                     a.vnorm_out[(static_cast<int64_t>(b) * H + h) * a.nb + i] =
-                        static_cast<float>(nacc * inv_cnt * x.scale);
+                        static_cast<float>(nacc * inv_cnt * scale);
                 }
             }
         } else {
+            if constexpr (DT != 1) {
 #pragma unroll
-            for (int e = 0; e < V; ++e) red[threadIdx.x][e] = acc[e];
+                for (int e = 0; e < V; ++e) red[threadIdx.x][e] = acc[e];
+            }
             red[threadIdx.x][V] = nacc;
             __syncthreads();
             if (live && tg == 0) {
@@ -219,10 +298,10 @@ __global__ void __launch_bounds__(kPoolThreads, 2) pool_kernel(const PoolArgs a)
                 if (!is_v) {
 #pragma unroll
                     for (int e = 0; e < V; ++e)
-                        store_split(a, which, o + e, static_cast<float>(red[threadIdx.x][e] * inv_cnt * x.scale));
+                        store_split(a, which, o + e, static_cast<float>(red[threadIdx.x][e] * inv_cnt * scale));
                 } else if (c0 == 0) {
                     a.vnorm_out[(static_cast<int64_t>(b) * H + h) * a.nb + i] =
-                        static_cast<float>(red[threadIdx.x][V] * inv_cnt * x.scale);
+                        static_cast<float>(red[threadIdx.x][V] * inv_cnt * scale);
                 }
             }
         }
