@@ -110,6 +110,14 @@ def bsa_tpd_budget(nb: int, density: float, tpd_decay: float = 0.5):
     return k[:nb], int(tot)
 
 
+def tpd_kstar(nb: int, density: float, tpd_decay: float = 0.5) -> int:
+    """K*, the TPD budget total of a sequence of nb blocks (bsa_tpd_budget with k_out = NULL)."""
+    tot = lib().bsa_tpd_budget(nb, float(density), float(tpd_decay), None)
+    if tot < 0:
+        raise BsaError(1, "invalid TPD arguments")
+    return int(tot)
+
+
 def bsa_score_workspace_bytes(B, Hq, Hkv, nb, d) -> int:
     return int(lib().bsa_score_workspace_bytes(B, Hq, Hkv, nb, d))
 
@@ -154,7 +162,7 @@ def stem_select(scores, nb_per_seq, density: float, tpd_decay: float = 0.5, row_
     B, Hq, nbs, _ = scores.shape
     nbp = torch.tensor(list(nb_per_seq), dtype=torch.int32)
     if max_k is None:
-        max_k = max(bsa_tpd_budget(int(n), density, tpd_decay)[1] for n in nbp)
+        max_k = max(tpd_kstar(int(n), density, tpd_decay) for n in nbp)
     if row_ptr is None:
         row_ptr = torch.empty(B, nbs + 1, dtype=torch.int32, device=scores.device)
     if col_idx is None:

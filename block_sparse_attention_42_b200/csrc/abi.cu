@@ -189,8 +189,9 @@ using namespace bsa;
 extern "C" {
 
 int64_t bsa_tpd_budget(int32_t nb, double density, double tpd_decay, int32_t* k_out) {
-    if (!k_out || !tpd_args_ok(nb, density, tpd_decay)) return -1;
+    if (!tpd_args_ok(nb, density, tpd_decay)) return -1;
     const int64_t kstar = tpd_kstar(nb, density);
+    if (!k_out) return kstar;
     const bool half = tpd_decay == 0.5;
     auto share = [&](double c, int i) -> int64_t {
         const double n = static_cast<double>(i + 1), m = i == 0 ? 1.0 : 2.0;

@@ -26,21 +26,20 @@ namespace {
 
 constexpr int kBudgetThreads = 1024;
 constexpr int kRowsPerThread = kMaxBlocks / kBudgetThreads;  // 2
+static_assert(kMaxBlocks <= 2048, "the leftover search takes row indices below 2^11");
 
-__device__ __forceinline__ long long block_sum_i64(long long v, long long* red) {
+// Sum of v over the CTA with one barrier: the per-warp sums go to red[par] (the buffer
+// alternates between calls, so a call's writes cannot race a slower thread's reads of the call
+// before), then every warp adds up all warp sums itself, in the same order.
+__device__ __forceinline__ long long block_sum_i64(long long v, long long (*red)[32], int& par) {
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
     const int w = threadIdx.x / 32, l = threadIdx.x % 32;
+    if (l == 0) red[par][w] = v;
     __syncthreads();
-    if (l == 0) red[w] = v;
-    __syncthreads();
-    long long t = 0;
-    if (threadIdx.x < 32) {
-        t = threadIdx.x < blockDim.x / 32 ? red[threadIdx.x] : 0;
-        for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xFFFFFFFFu, t, o);
-        if (threadIdx.x == 0) red[32] = t;
-    }
-    __syncthreads();
-    return red[32];
+    long long t = l < static_cast<int>(blockDim.x / 32) ? red[par][l] : 0;
+    for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xFFFFFFFFu, t, o);
+    par ^= 1;
+    return t;
 }
 
 __device__ __forceinline__ long long fixed_share(double c, double w, double n, double m) {
@@ -52,8 +51,9 @@ __device__ __forceinline__ long long fixed_share(double c, double w, double n, d
 
 __global__ void __launch_bounds__(kBudgetThreads) tpd_budget_kernel(const SelectSeqs seqs, int decay_half,
                                                                     int32_t* __restrict__ row_ptr, int nbs) {
-    __shared__ long long red[33];
+    __shared__ long long red[2][32];
     __shared__ int wsum[33];
+    int par = 0;
     const int b = blockIdx.x;
     const int nb = seqs.nb[b];
     const long long kstar = seqs.kstar[b];
@@ -78,7 +78,7 @@ __global__ void __launch_bounds__(kBudgetThreads) tpd_budget_kernel(const Select
             const int i = threadIdx.x * kRowsPerThread + r;
             if (valid[r]) part += fixed_share(mid, w[r], static_cast<double>(i + 1), i == 0 ? 1.0 : 2.0);
         }
-        const long long tot = block_sum_i64(part, red);
+        const long long tot = block_sum_i64(part, red, par);
         if (tot >= target)
             hi = mid;
         else
@@ -101,16 +101,23 @@ __global__ void __launch_bounds__(kBudgetThreads) tpd_budget_kernel(const Select
             key[r] = (static_cast<unsigned long long>(F & 0xFFFFFFFFll) << 32) |
                      (0xFFFFFFFFull - static_cast<unsigned long long>(i));
     }
-    const long long R = kstar - block_sum_i64(whole, red);
+    const long long R = kstar - block_sum_i64(whole, red, par);
     if (R > 0) {
-        // The R-th largest key (keys are distinct) by a bitwise search on its value.
+        // The R-th largest key (keys are distinct) by a bitwise search on its value.  Bits
+        // 31..11 are set in every eligible key (row indices are below 2048), so once the
+        // fraction is found they are set without a count.
         unsigned long long thr = 0;
         for (int bit = 63; bit >= 0; --bit) {
+            if (bit == 31) {
+                thr |= 0xFFFFF800ull;
+                bit = 11;
+                continue;
+            }
             const unsigned long long cand = thr | (1ull << bit);
             long long cnt = 0;
 #pragma unroll
             for (int r = 0; r < kRowsPerThread; ++r) cnt += key[r] >= cand ? 1 : 0;
-            if (block_sum_i64(cnt, red) >= R) thr = cand;
+            if (block_sum_i64(cnt, red, par) >= R) thr = cand;
         }
 #pragma unroll
         for (int r = 0; r < kRowsPerThread; ++r)

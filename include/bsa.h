@@ -73,8 +73,9 @@ typedef struct {
 /* TPD budget of one sequence with nb query blocks, computed on the HOST (the same rule the
  * select kernel runs on the device): k_out[i] (host array of nb) receives the number of KV
  * blocks kept by query block i; returns their sum K*, or -1 for invalid arguments.
- * density in (0, 1]; tpd_decay in {0 (uniform), 0.5 (keep ratio ~ (i+1)^-1/2)}.  Use it to
- * size col_idx (max_k >= K* of every sequence).  [cn486 page, §3.1 TPD.] */
+ * density in (0, 1]; tpd_decay in {0 (uniform), 0.5 (keep ratio ~ (i+1)^-1/2)}.  With
+ * k_out = NULL only K* is computed (no per-row budget, O(1)).  Use it to size col_idx
+ * (max_k >= K* of every sequence).  [cn486 page, §3.1 TPD.] */
 int64_t bsa_tpd_budget(int32_t nb, double density, double tpd_decay, int32_t* k_out);
 
 /* Bytes of device workspace stem_score needs for B sequences of nb blocks. */

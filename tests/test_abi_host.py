@@ -40,6 +40,8 @@ def test_host_budget_equals_oracle_exhaustive(lib, orc):
                 k, tot = binding.bsa_tpd_budget(nb, density, decay)
                 ko, toto = orc.tpd_budget(nb, density, decay)
                 assert tot == toto and np.array_equal(k.numpy(), ko), (nb, density, decay)
+                # k_out = NULL: the total alone
+                assert binding.tpd_kstar(nb, density, decay) == toto, (nb, density, decay)
 
 
 def test_host_budget_rejects_bad_args(lib):
@@ -47,6 +49,8 @@ def test_host_budget_rejects_bad_args(lib):
     assert lib.bsa_tpd_budget(0, 0.5, 0.5, k) == -1
     assert lib.bsa_tpd_budget(8, 0.0, 0.5, k) == -1
     assert lib.bsa_tpd_budget(8, 0.5, 0.25, k) == -1
+    assert lib.bsa_tpd_budget(0, 0.5, 0.5, None) == -1
+    assert lib.bsa_tpd_budget(8, 1.5, 0.5, None) == -1
 
 
 def _t(ptr=0x10000, dtype=0, st=1024, sh=128, sb=1 << 20, scale=1.0):
