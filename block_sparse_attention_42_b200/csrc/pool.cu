@@ -10,9 +10,9 @@
 // row is read once with fully coalesced 16-byte loads.  Sums are kept in fp64 (cheap here:
 // the kernel waits on HBM) so the pooled means carry only the final fp32 rounding.  What
 // bounds it is the number of 16-byte loads in flight per SM, so the E4M3 instantiation keeps
-// its fp64 sums in shared memory and its registers at 64 per thread, for four CTAs per SM.  Each Q/K
-// mean is written as two fp32 arrays, a TF32-exact high part and the remainder, which the
-// tensor-core score GEMM consumes directly (score_tc.cu).
+// its fp64 sums in shared memory and its registers at 64 per thread, for four CTAs per SM.
+// Each Q/K mean is written as two fp32 arrays, a TF32-exact high part and the remainder,
+// which the tensor-core score GEMM consumes directly (score_tc.cu).
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 
@@ -39,44 +39,17 @@ struct Elem<0> {  // bf16
     }
 };
 template <>
-struct Elem<1> {  // e4m3
+struct Elem<1> {  // e4m3: summed through the f16x2 path in pool_kernel, no float decode
     static constexpr int kVec = 16;
-    // Exact decode with integer ops and one multiply (no conversion instructions): the code's
-    // 7 exponent/mantissa bits placed at fp32 bits 26..20 (sign at 31) read as 2^(e-127) *
-    // (1 + m/8), or as the denormal m/8 * 2^-126 when e = 0; times 2^120 that is the E4M3
-    // value (bias 7), subnormals included.  (Denormals are kept: no flush-to-zero here.)
-    __device__ static void decode(const uint4& raw, float (&f)[16]) {
-        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const uint32_t b = (w[i] >> (8 * q)) & 0xFFu;
-                f[4 * i + q] = __uint_as_float(((b & 0x80u) << 24) | ((b & 0x7Fu) << 20)) * 0x1p120f;
-            }
-        }
-        // The NaN codes (x111_1111) would read as +-480 above: a word holding one has a byte
-        // whose low 7 bits + 1 carry into bit 7.
-        uint32_t nan_any = 0;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) nan_any |= ((w[i] & 0x7F7F7F7Fu) + 0x01010101u) & 0x80808080u;
-        if (nan_any) {
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-                if (((w[i / 4] >> (8 * (i % 4))) & 0x7Fu) == 0x7Fu) f[i] = __uint_as_float(0x7FC00000u);
-        }
-    }
 };
-// Four E4M3 codes of w -> two f16x2 words holding each code's value times 2^-8, exactly (an
-// E4M3 code read as f16 with its 7 exponent/mantissa bits moved to f16 bits 13..7: the
-// exponent bias goes from 7 to 15, subnormals map to subnormals).  h01 holds codes 0 (low
-// half) and 1, h23 codes 2 and 3.  The NaN codes come out finite (+-480 * 2^-8); callers test
-// for them separately.
-__device__ __forceinline__ void e4m3x4_to_f16x2(uint32_t w, uint32_t& h01, uint32_t& h23) {
-    const uint32_t x01 = __byte_perm(w, 0u, 0x1404);  // code 1 << 24 | code 0 << 8
-    const uint32_t x23 = __byte_perm(w, 0u, 0x3424);  // code 3 << 24 | code 2 << 8
-    h01 = (x01 & 0x80008000u) | ((x01 >> 1) & 0x3F803F80u);
-    h23 = (x23 & 0x80008000u) | ((x23 >> 1) & 0x3F803F80u);
+// Two E4M3 codes (low 16 bits of w >> 16*half) -> f16x2, exact; NaN codes give NaN.
+__device__ __forceinline__ uint32_t cvt_e4m3x2(uint32_t w, int half) {
+    uint32_t d;
+    if (half == 0)
+        asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, l;\n\t}" : "=r"(d) : "r"(w));
+    else
+        asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, h;\n\t}" : "=r"(d) : "r"(w));
+    return d;
 }
 
 // c + the low / high f16 half of h2, rounded once to fp32 (sm_100 mixed-precision add).
@@ -145,9 +118,7 @@ __global__ void __launch_bounds__(kPoolThreads, DT == 1 ? 4 : 2) pool_kernel(con
     const int t_lo = i * a.block;
     const int t_hi = min(a.N, t_lo + a.block);
     const double inv_cnt = 1.0 / static_cast<double>(t_hi - t_lo);
-    // E4M3 sums are of the values times 2^-8 (below); the final scale puts the 2^8 back, with
-    // the same roundings as unscaled sums would get.
-    const double scale = static_cast<double>(x.scale) * (DT == 1 ? 256.0 : 1.0);
+    const double scale = static_cast<double>(x.scale);
     const bool is_v = (which == 2);
 
     __shared__ double red[kPoolThreads][V + 1];
@@ -173,8 +144,9 @@ __global__ void __launch_bounds__(kPoolThreads, DT == 1 ? 4 : 2) pool_kernel(con
         }
         double nacc = 0.0;
         // E4M3: values are multiples of 2^-9 below 2^9, so any sum of up to 64 of them is exact
-        // in fp32 (also after scaling by 2^-8); such partial sums are flushed into the fp64
-        // sums every kFlush batches.
+        // in fp32; such partial sums are flushed into the fp64 sums every kFlush batches.  Each
+        // pair of codes becomes an f16x2 word (a hardware conversion, exact, NaN codes to NaN)
+        // whose halves are added into the fp32 sums directly (sm_100 mixed-precision add).
         float facc[V];
 #pragma unroll
         for (int e = 0; e < V; ++e) facc[e] = 0.f;
@@ -202,34 +174,16 @@ __global__ void __launch_bounds__(kPoolThreads, DT == 1 ? 4 : 2) pool_kernel(con
 #pragma unroll
             for (int u = 0; u < kBatch; ++u) {
                 if constexpr (DT == 1) {
-                    // Sums of the codes' values times 2^-8 (f16 halves added into fp32: exact, as
-                    // above, since the scaling is a power of two); the 2^8 goes into the final
-                    // scale.  A vector holding a NaN code takes the float decode, which gives NaN.
                     const uint32_t w[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
-                    uint32_t nan_any = 0;
+                    float ss = 0.f;  // V: fp32 sum of squares (relative error ~1e-7 in the norm)
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) nan_any |= ((w[q] & 0x7F7F7F7Fu) + 0x01010101u) & 0x80808080u;
-                    float ss = 0.f;  // V: fp32 sum of squares, times 2^-16 (relative error ~1e-7)
-                    if (nan_any == 0) {
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            uint32_t h01, h23;
-                            e4m3x4_to_f16x2(w[q], h01, h23);
-                            facc[4 * q + 0] = add_f16lo(h01, facc[4 * q + 0]);
-                            facc[4 * q + 1] = add_f16hi(h01, facc[4 * q + 1]);
-                            facc[4 * q + 2] = add_f16lo(h23, facc[4 * q + 2]);
-                            facc[4 * q + 3] = add_f16hi(h23, facc[4 * q + 3]);
-                            if (is_v) ss = sq_f16hi(h23, sq_f16lo(h23, sq_f16hi(h01, sq_f16lo(h01, ss))));
-                        }
-                    } else {
-                        float f[V];
-                        Elem<1>::decode(raw[u], f);
-#pragma unroll
-                        for (int e = 0; e < V; ++e) {
-                            const float fs = f[e] * 0x1p-8f;
-                            facc[e] += fs;
-                            ss = fmaf(fs, fs, ss);
-                        }
+                    for (int q = 0; q < 4; ++q) {
+                        const uint32_t h01 = cvt_e4m3x2(w[q], 0), h23 = cvt_e4m3x2(w[q], 1);
+                        facc[4 * q + 0] = add_f16lo(h01, facc[4 * q + 0]);
+                        facc[4 * q + 1] = add_f16hi(h01, facc[4 * q + 1]);
+                        facc[4 * q + 2] = add_f16lo(h23, facc[4 * q + 2]);
+                        facc[4 * q + 3] = add_f16hi(h23, facc[4 * q + 3]);
+                        if (is_v) ss = sq_f16hi(h23, sq_f16lo(h23, sq_f16hi(h01, sq_f16lo(h01, ss))));
                     }
                     if (is_v) {
                         for (int o = 1; o < vec_per_head; o <<= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
