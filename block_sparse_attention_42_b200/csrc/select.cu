@@ -24,20 +24,25 @@
 namespace bsa {
 namespace {
 
-constexpr int kBudgetThreads = 1024;
-constexpr int kRowsPerThread = kMaxBlocks / kBudgetThreads;  // 2
+constexpr int kBudgetThreads = 256;
+constexpr int kRowsPerThread = kMaxBlocks / kBudgetThreads;  // 8
 static_assert(kMaxBlocks <= 2048, "the leftover search takes row indices below 2^11");
 
-// Sum of v over the CTA with one barrier: the per-warp sums go to red[par] (the buffer
-// alternates between calls, so a call's writes cannot race a slower thread's reads of the call
-// before), then every warp adds up all warp sums itself, in the same order.
+// Sum of v over the CTA with one barrier, for 0 <= v < 2^46 (a thread's fixed-point shares:
+// at most 8 rows of at most 2^43 each).  Each warp adds the low 22 and the high 24 bits of v
+// separately with one warp reduction each (sums below 2^27 and 2^29: no overflow), lane 0
+// stores the warp's sum in red[par] (the buffer alternates between calls, so a call's writes
+// cannot race a slower thread's reads of the call before), and every thread adds up the warp
+// sums in the same order.
 __device__ __forceinline__ long long block_sum_i64(long long v, long long (*red)[32], int& par) {
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
-    const int w = threadIdx.x / 32, l = threadIdx.x % 32;
-    if (l == 0) red[par][w] = v;
+    const uint32_t lo = __reduce_add_sync(0xFFFFFFFFu, static_cast<uint32_t>(v & 0x3FFFFF));
+    const uint32_t hi = __reduce_add_sync(0xFFFFFFFFu, static_cast<uint32_t>(v >> 22));
+    const int w = threadIdx.x / 32;
+    if (threadIdx.x % 32 == 0) red[par][w] = (static_cast<long long>(hi) << 22) + lo;
     __syncthreads();
-    long long t = l < static_cast<int>(blockDim.x / 32) ? red[par][l] : 0;
-    for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xFFFFFFFFu, t, o);
+    long long t = 0;
+#pragma unroll
+    for (int q = 0; q < kBudgetThreads / 32; ++q) t += red[par][q];
     par ^= 1;
     return t;
 }
