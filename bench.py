@@ -526,7 +526,9 @@ def main():
             # per SM (measured with a throughput probe on this machine), so the peak is
             # 16 x SMs x the median SM clock sampled during the timed steps.
             "roofline_mufu": mufu_roofline(res, device),
-            "gpu_launches": 5 * args.steps,
+            # pool, score, TPD budget, one select launch per row-length class present
+            # (query blocks in [0, 256), [256, 512), [512, 1024), [1024, 2048)), attention
+            "gpu_launches": (4 + sum(1 for lo in (0, 256, 512, 1024) if res["nb"] > lo)) * args.steps,
             "clocks": res["clocks"],
         }
         if "dense_ms" in res:

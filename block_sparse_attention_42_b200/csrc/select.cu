@@ -164,6 +164,12 @@ __global__ void __launch_bounds__(kBudgetThreads) tpd_budget_kernel(const Select
 
 constexpr int kSelWarps = 8;
 
+// Query blocks of a sequence with nb blocks that fall in [i_lo, i_hi).
+__host__ __device__ __forceinline__ int class_rows(int nb, int i_lo, int i_hi) {
+    const int hi = nb < i_hi ? nb : i_hi;
+    return hi > i_lo ? hi - i_lo : 0;
+}
+
 __device__ __forceinline__ uint32_t order_key(float s) {
     if (s != s) s = -INFINITY;   // NaN ranks as -inf
     if (s == 0.f) s = 0.f;       // -0 and +0 tie
@@ -171,11 +177,13 @@ __device__ __forceinline__ uint32_t order_key(float s) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// Rows whose query block i lies in [i_lo, i_hi) (i_hi <= 32 * MAXPL), so that each launch is
+// compiled for the longest row it sees and short rows issue no work for positions they lack.
 template <int MAXPL>
 __global__ void __launch_bounds__(kSelWarps * 32) select_kernel(const float* __restrict__ S, const SelectSeqs seqs,
                                                                 int Hq, int nbs, const int32_t* __restrict__ row_ptr,
                                                                 int32_t* __restrict__ col_idx, int64_t max_k,
-                                                                long long total_rows) {
+                                                                long long total_rows, int i_lo, int i_hi) {
     __shared__ uint32_t hist_all[kSelWarps][256];
     const int lane = threadIdx.x % 32, wid = threadIdx.x / 32;
     uint32_t* hist = hist_all[wid];
@@ -186,12 +194,12 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_kernel(const float* __r
         // Row order: sequence-major, then longest rows (largest i) first.
         long long rr = row;
         int b = 0;
-        while (rr >= static_cast<long long>(seqs.nb[b]) * Hq) {
-            rr -= static_cast<long long>(seqs.nb[b]) * Hq;
+        while (rr >= static_cast<long long>(class_rows(seqs.nb[b], i_lo, i_hi)) * Hq) {
+            rr -= static_cast<long long>(class_rows(seqs.nb[b], i_lo, i_hi)) * Hq;
             ++b;
         }
         const int nb = seqs.nb[b];
-        const int i = nb - 1 - static_cast<int>(rr / Hq);
+        const int i = min(nb, i_hi) - 1 - static_cast<int>(rr / Hq);
         const int h = static_cast<int>(rr % Hq);
         const int32_t* rp = row_ptr + static_cast<int64_t>(b) * (nbs + 1);
         const int start = rp[i];
@@ -306,11 +314,15 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_kernel(const float* __r
 
 template <int MAXPL>
 cudaError_t launch_sel(const float* scores, const SelectSeqs& seqs, int Hq, int nbs, const int32_t* row_ptr,
-                       int32_t* col_idx, int64_t max_k, long long total, cudaStream_t s) {
+                       int32_t* col_idx, int64_t max_k, cudaStream_t s) {
+    const int i_lo = MAXPL == 8 ? 0 : 16 * MAXPL, i_hi = 32 * MAXPL;
+    long long total = 0;
+    for (int b = 0; b < seqs.B; ++b) total += static_cast<long long>(class_rows(seqs.nb[b], i_lo, i_hi)) * Hq;
+    if (total == 0) return cudaSuccess;
     long long blocks = (total + kSelWarps - 1) / kSelWarps;
     if (blocks > 148 * 16) blocks = 148 * 16;
     select_kernel<MAXPL><<<static_cast<unsigned>(blocks), kSelWarps * 32, 0, s>>>(scores, seqs, Hq, nbs, row_ptr,
-                                                                                  col_idx, max_k, total);
+                                                                                  col_idx, max_k, total, i_lo, i_hi);
     return cudaGetLastError();
 }
 
@@ -321,16 +333,12 @@ cudaError_t launch_select(const float* scores, const SelectSeqs& seqs, int Hq, i
     tpd_budget_kernel<<<seqs.B, kBudgetThreads, 0, s>>>(seqs, decay_half ? 1 : 0, row_ptr, nb_stride);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    int nbmax = 0;
-    long long total = 0;
-    for (int b = 0; b < seqs.B; ++b) {
-        nbmax = seqs.nb[b] > nbmax ? seqs.nb[b] : nbmax;
-        total += static_cast<long long>(seqs.nb[b]) * Hq;
-    }
-    if (nbmax <= 256) return launch_sel<8>(scores, seqs, Hq, nb_stride, row_ptr, col_idx, max_k, total, s);
-    if (nbmax <= 512) return launch_sel<16>(scores, seqs, Hq, nb_stride, row_ptr, col_idx, max_k, total, s);
-    if (nbmax <= 1024) return launch_sel<32>(scores, seqs, Hq, nb_stride, row_ptr, col_idx, max_k, total, s);
-    return launch_sel<64>(scores, seqs, Hq, nb_stride, row_ptr, col_idx, max_k, total, s);
+    // One launch per row-length class, longest rows first: i in [1024, 2048), [512, 1024),
+    // [256, 512), [0, 256).
+    if ((e = launch_sel<64>(scores, seqs, Hq, nb_stride, row_ptr, col_idx, max_k, s)) != cudaSuccess) return e;
+    if ((e = launch_sel<32>(scores, seqs, Hq, nb_stride, row_ptr, col_idx, max_k, s)) != cudaSuccess) return e;
+    if ((e = launch_sel<16>(scores, seqs, Hq, nb_stride, row_ptr, col_idx, max_k, s)) != cudaSuccess) return e;
+    return launch_sel<8>(scores, seqs, Hq, nb_stride, row_ptr, col_idx, max_k, s);
 }
 
 }  // namespace bsa
