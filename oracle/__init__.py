@@ -70,6 +70,8 @@ def _load():
     lib.orc_select.restype = ctypes.c_int
     lib.orc_attention_rows.argtypes = [T, T, T, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                        ctypes.c_int, P, ctypes.c_int, P, i64, f64, P, i64, P, P]
+    lib.orc_attention_rows_mask.argtypes = [T, T, T, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                            ctypes.c_int, P, i64, f64, P, i64, P, P]
     lib.orc_effective_flop.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, P,
                                        ctypes.c_int, P, i64, ctypes.c_int]
     lib.orc_effective_flop.restype = f64
@@ -201,6 +203,20 @@ def attention_rows(q: View, k: View, v: View, N, Hq, Hkv, D, bs, row_ptr, col_id
     _load().orc_attention_rows(ctypes.byref(q.struct), ctypes.byref(k.struct), ctypes.byref(v.struct),
                                N, Hq, Hkv, D, bs, _ptr(row_ptr), row_ptr.shape[-1], _ptr(col_idx),
                                col_idx.shape[-1], float(tau), _ptr(rows), n, _ptr(out), _ptr(lse))
+    return out, lse
+
+
+def attention_rows_mask(q: View, k: View, v: View, N, Hq, Hkv, D, bs, mask, tau, rows):
+    """O and LSE of the requested (b, h, t) rows with the selection as a block mask
+    [B, Hq, nb, >= nb] (uint8; nonzero = kept), fp64.  Empty rows: O = 0, LSE = -inf."""
+    mask = np.ascontiguousarray(np.asarray(mask, dtype=np.uint8))
+    rows = _c(rows, np.int64).reshape(-1, 3)
+    n = rows.shape[0]
+    out = np.empty((n, D), np.float64)
+    lse = np.empty((n,), np.float64)
+    _load().orc_attention_rows_mask(ctypes.byref(q.struct), ctypes.byref(k.struct), ctypes.byref(v.struct),
+                                    N, Hq, Hkv, D, bs, _ptr(mask), mask.shape[-1], float(tau), _ptr(rows), n,
+                                    _ptr(out), _ptr(lse))
     return out, lse
 
 

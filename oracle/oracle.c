@@ -32,6 +32,9 @@
  *   orc_select          pinned: brute-force full sort; kept scores dominate dropped ones.
  *   orc_attention_rows  pinned: density 1 == library dense causal SDPA (fp64); skipped
  *                       blocks' contents are irrelevant; single-key closed form.
+ *   orc_attention_rows_mask  pinned: an all-ones mask == library dense causal SDPA; a
+ *                       diagonal-only mask == library SDPA over the block's own keys; an
+ *                       empty row gives 0 / -inf; entries above the diagonal are ignored.
  */
 #include <math.h>
 #include <stdint.h>
@@ -401,6 +404,59 @@ void orc_attention_rows(const orc_tensor* q, const orc_tensor* k, const orc_tens
             if (lse) lse[r] = m + log(z);
         }
         free(allowed);
+        free(logit);
+        free(qrow);
+    }
+}
+
+/* The same attention with the selection given as a block mask instead of lists
+ * [P1 §二.2.2: HPC-BSA receives the selection as a block mask; a skipped block is a block of
+ * -inf scores].  mask is [B][Hq][nb][mask_stride] bytes; the allowed keys of query token t
+ * (block i) of head h are A(t) = {s <= t : mask[b][h][i][block(s)] != 0}.  A row with A(t)
+ * empty has no softmax; its output is taken as O = 0 and lse = -inf (the convention of
+ * softmax over an empty set used by attention kernels).  The mask is read per key. */
+void orc_attention_rows_mask(const orc_tensor* q, const orc_tensor* k, const orc_tensor* v, int N,
+                             int Hq, int Hkv, int D, int bs, const uint8_t* mask, int64_t mask_stride,
+                             double tau, const int64_t* rows, int64_t n_rows, double* out /* [n_rows][D] */,
+                             double* lse /* [n_rows] */) {
+    int G = Hq / Hkv;
+    int64_t nb = (N + bs - 1) / bs;
+#pragma omp parallel
+    {
+        double* logit = (double*)malloc(sizeof(double) * (size_t)N);
+        double* qrow = (double*)malloc(sizeof(double) * (size_t)D);
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t r = 0; r < n_rows; ++r) {
+            int64_t b = rows[3 * r], h = rows[3 * r + 1], t = rows[3 * r + 2];
+            int64_t hk = h / G;
+            const uint8_t* mrow = &mask[((b * Hq + h) * nb + t / bs) * mask_stride];
+            for (int c = 0; c < D; ++c) qrow[c] = load_elem(q, b, t, h, c);
+            double m = -INFINITY;
+            int any = 0;
+            for (int64_t s = 0; s <= t; ++s) {
+                if (mrow[s / bs] == 0) continue;
+                double dot = 0.0;
+                for (int c = 0; c < D; ++c) dot += qrow[c] * load_elem(k, b, s, hk, c);
+                logit[s] = tau * dot;
+                if (logit[s] > m) m = logit[s];
+                any = 1;
+            }
+            double* o = &out[r * D];
+            for (int c = 0; c < D; ++c) o[c] = 0.0;
+            if (!any) {
+                if (lse) lse[r] = -INFINITY;
+                continue;
+            }
+            double z = 0.0;
+            for (int64_t s = 0; s <= t; ++s) {
+                if (mrow[s / bs] == 0) continue;
+                double w = exp(logit[s] - m);
+                z += w;
+                for (int c = 0; c < D; ++c) o[c] += w * load_elem(v, b, s, hk, c);
+            }
+            for (int c = 0; c < D; ++c) o[c] /= z;
+            if (lse) lse[r] = m + log(z);
+        }
         free(logit);
         free(qrow);
     }

@@ -312,6 +312,113 @@ def test_single_key_closed_form(orc):
     assert lse[0] == pytest.approx(0.7 * float(q[0, 0, 0] @ k[0, 0, 0]), rel=1e-15)
 
 
+# ----------------------------------------------------------------------------- block-mask input
+
+
+def test_mask_all_ones_equals_library_causal_sdpa(orc):
+    """An all-ones block mask (above the diagonal too) is dense causal attention."""
+    w = inputs.Workload("pin", 2, 4, 2, 45, 16, 8, "fp32", 1.0, "stem", 96)
+    d = inputs.make_inputs(w)
+    q, k, v = d["q"].double(), d["k"].double(), d["v"].double()
+    B, N, Hq, Hkv, D, bs = 2, 45, 4, 2, 16, 8
+    nb = (N + bs - 1) // bs
+    mask = np.ones((B, Hq, nb, 16), np.uint8)
+    tau = 1 / math.sqrt(D)
+    out, lse = orc.attention_rows_mask(orc.view(q), orc.view(k), orc.view(v), N, Hq, Hkv, D, bs, mask, tau,
+                                       _all_rows(B, Hq, N))
+    G = Hq // Hkv
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        q.transpose(1, 2), k.repeat_interleave(G, 2).transpose(1, 2), v.repeat_interleave(G, 2).transpose(1, 2),
+        is_causal=True, scale=tau).transpose(1, 2)
+    ref = ref.permute(0, 2, 1, 3).reshape(-1, D).numpy()
+    np.testing.assert_allclose(out, ref, rtol=1e-12, atol=1e-12)
+    logits = torch.einsum("bthd,bshd->bhts", q, k.repeat_interleave(G, 2)) * tau
+    causal = torch.ones(N, N, dtype=torch.bool).tril()
+    ref_lse = torch.logsumexp(logits.masked_fill(~causal, float("-inf")), -1).reshape(-1).numpy()
+    np.testing.assert_allclose(lse, ref_lse, rtol=1e-12, atol=1e-12)
+
+
+def test_mask_diagonal_only_equals_sdpa_within_the_block(orc):
+    """Only the diagonal block kept: each block is causal attention over its own keys."""
+    rng = np.random.default_rng(11)
+    B, N, Hq, Hkv, D, bs = 1, 37, 2, 1, 8, 8
+    nb = (N + bs - 1) // bs
+    q = rng.standard_normal((B, N, Hq, D)); k = rng.standard_normal((B, N, Hkv, D)); v = rng.standard_normal((B, N, Hkv, D))
+    mask = np.zeros((B, Hq, nb, 16), np.uint8)
+    for i in range(nb):
+        mask[:, :, i, i] = 1
+    tau = 0.41
+    out, _ = orc.attention_rows_mask(orc.view(q), orc.view(k), orc.view(v), N, Hq, Hkv, D, bs, mask, tau,
+                                     _all_rows(B, Hq, N))
+    out = out.reshape(Hq, N, D)
+    for h in range(Hq):
+        for i in range(nb):
+            lo, hi = i * bs, min(N, (i + 1) * bs)
+            ref = torch.nn.functional.scaled_dot_product_attention(
+                torch.from_numpy(q[0, lo:hi, h]), torch.from_numpy(k[0, lo:hi, 0]), torch.from_numpy(v[0, lo:hi, 0]),
+                is_causal=True, scale=tau)
+            np.testing.assert_allclose(out[h, lo:hi], ref.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_mask_empty_row_and_upper_triangle(orc):
+    """A row keeping nothing gives O = 0, LSE = -inf; entries above the diagonal change nothing."""
+    rng = np.random.default_rng(12)
+    B, N, Hq, Hkv, D, bs = 1, 32, 1, 1, 4, 8
+    nb = 4
+    q = rng.standard_normal((B, N, Hq, D)); k = rng.standard_normal((B, N, Hkv, D)); v = rng.standard_normal((B, N, Hkv, D))
+    mask = np.zeros((B, Hq, nb, 16), np.uint8)
+    mask[0, 0, 2, :3] = [1, 0, 1]                            # row 2: blocks 0 and 2
+    rows = _all_rows(B, Hq, N)
+    out, lse = orc.attention_rows_mask(orc.view(q), orc.view(k), orc.view(v), N, Hq, Hkv, D, bs, mask, 0.5, rows)
+    empty = [t for t in range(N) if t // bs != 2]
+    assert np.all(out[empty] == 0.0) and np.all(np.isneginf(lse[empty]))
+    upper = mask.copy()
+    upper[0, 0, 0, 1:] = 7                                   # above the diagonal
+    upper[0, 0, 2, 3] = 1
+    out2, lse2 = orc.attention_rows_mask(orc.view(q), orc.view(k), orc.view(v), N, Hq, Hkv, D, bs, upper, 0.5, rows)
+    assert np.array_equal(out, out2) and np.array_equal(lse, lse2)
+    # row 2 against the library with the token mask written out
+    tm = torch.zeros(bs, N, dtype=torch.bool)
+    tm[:, 0:8] = True
+    tm[:, 16:24] = True
+    tm &= torch.ones(N, N, dtype=torch.bool).tril()[16:24]
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q[0, 16:24, 0]), torch.from_numpy(k[0, :, 0]), torch.from_numpy(v[0, :, 0]),
+        attn_mask=tm, scale=0.5)
+    np.testing.assert_allclose(out[16:24], ref.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_mask_per_head_equals_library_masked_sdpa(orc):
+    """Random, different masks per query head (GQA): each head against the library's SDPA with
+    the token mask written out; rows that keep nothing are 0 / -inf."""
+    rng = np.random.default_rng(13)
+    B, N, Hq, Hkv, D, bs = 1, 45, 4, 2, 8, 8
+    nb = (N + bs - 1) // bs
+    q = rng.standard_normal((B, N, Hq, D)); k = rng.standard_normal((B, N, Hkv, D)); v = rng.standard_normal((B, N, Hkv, D))
+    mask = (rng.random((B, Hq, nb, 16)) < 0.4).astype(np.uint8)
+    mask[0, 1, 3, :] = 0                                     # an empty row
+    tau = 0.29
+    out, lse = orc.attention_rows_mask(orc.view(q), orc.view(k), orc.view(v), N, Hq, Hkv, D, bs, mask, tau,
+                                       _all_rows(B, Hq, N))
+    out, lse = out.reshape(Hq, N, D), lse.reshape(Hq, N)
+    G = Hq // Hkv
+    causal = torch.ones(N, N, dtype=torch.bool).tril()
+    for h in range(Hq):
+        tm = torch.zeros(N, N, dtype=torch.bool)
+        for i in range(nb):
+            for j in range(nb):
+                if mask[0, h, i, j]:
+                    tm[i * bs:(i + 1) * bs, j * bs:(j + 1) * bs] = True
+        tm &= causal
+        live = tm.any(-1).numpy()
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(q[0, :, h]), torch.from_numpy(k[0, :, h // G]), torch.from_numpy(v[0, :, h // G]),
+            attn_mask=tm, scale=tau).numpy()
+        np.testing.assert_allclose(out[h][live], ref[live], rtol=1e-12, atol=1e-12)
+        assert np.all(out[h][~live] == 0.0) and np.all(np.isneginf(lse[h][~live]))
+    assert np.all(np.isneginf(lse[1, 24:32])) and np.all(out[1, 24:32] == 0.0)   # the emptied row
+
+
 def test_effective_flop_counts_pairs(orc):
     for N, bs in [(64, 8), (61, 8), (128, 64)]:
         nb = (N + bs - 1) // bs
