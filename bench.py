@@ -49,6 +49,7 @@ def parse():
                    help="query-head chunks per KV-head group in the pipelined end-to-end step (1 measured "
                         "fastest at fp8-128k: 56.0 ms vs 57.3 / 62.3 for 2 / 4)")
     p.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
+    p.add_argument("--no-mask", action="store_true", help="skip the block-mask input measurement")
     return p.parse_args()
 
 
@@ -272,6 +273,45 @@ def run_ours(args, rank, world, device):
         res["dense_ms"] = e0.elapsed_time(e1) / reps
         res["dense_flop"] = effective_flop(dense_rp, dense_ci, [N] * B, w.block, D)
         del dense_out, dense_ci
+
+    # Block-mask input (bsa_prefill_mask): the step's lists written as a [B, Hq, nb, nb] uint8
+    # mask (setup, untimed), then the mask -> lists kernel alone and the whole call, timed with
+    # events like the step.  Its output is the list path's bit for bit (tests/test_gpu_mask.py).
+    if not args.no_mask and rank == 0:
+        mask = bsa.block_mask_buffer(B, Hq, nb, device=device)
+        counts = (row_ptr[:, 1:] - row_ptr[:, :-1]).long()
+        for b in range(B):
+            rows = torch.repeat_interleave(torch.arange(nb, device=device), counts[b])
+            heads = torch.arange(Hq, device=device)[:, None].expand(Hq, rows.numel())
+            mask[b][heads, rows[None].expand(Hq, -1), col_idx[b, :, :rows.numel()].long()] = 1
+        mws = torch.empty(bsa.bsa_mask_workspace_bytes(B, Hq, nb), dtype=torch.uint8, device=device)
+        lrp = torch.empty(B, Hq, nb + 1, dtype=torch.int32, device=device)
+        lci = torch.empty(B, Hq, nb * (nb + 1) // 2, dtype=torch.int32, device=device)
+        mout = torch.empty_like(out)
+        bsa.bsa_mask_to_lists(mask, row_ptr=lrp, col_idx=lci)
+        bsa.bsa_prefill_mask(q, k, v, w.block, mask, out=mout, workspace=mws, **scale_kw)
+        torch.cuda.synchronize(device)
+        bsa.bsa_check_device_error(device)
+        same = bool(torch.equal(mout.view(torch.int16), out.view(torch.int16)))
+        reps = 3
+        e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        e0.record(stream)
+        for _ in range(reps):
+            bsa.bsa_mask_to_lists(mask, row_ptr=lrp, col_idx=lci)
+        e1.record(stream)
+        for _ in range(reps):
+            bsa.bsa_prefill_mask(q, k, v, w.block, mask, out=mout, workspace=mws, **scale_kw)
+        e2.record(stream)
+        torch.cuda.synchronize(device)
+        lists_ms = e0.elapsed_time(e1) / reps
+        # Algorithmic bytes of mask -> lists: each causal mask byte read once, the lists
+        # (sum of kept blocks) and row_ptr written once.
+        kept = int(counts.sum().item()) * Hq
+        mbytes = B * Hq * nb * (nb + 1) // 2 + 4 * kept + 4 * B * Hq * (nb + 1)
+        res["mask"] = {"prefill_mask_ms": e1.elapsed_time(e2) / reps, "mask_to_lists_ms": lists_ms,
+                       "mask_to_lists_gbs": mbytes / (lists_ms * 1e-3) / 1e9, "algorithmic_bytes": mbytes,
+                       "output_equals_list_path": same}
+        del mask, mws, lrp, lci, mout
 
     # End to end through the public API with host buffers: H2D of Q/K/V from pinned memory,
     # the step, D2H of the output, all inside the timed region.  The step is pipelined over
@@ -540,6 +580,12 @@ def main():
             line["e2e"] = {"value": whole_job_tflops(res["eff_flop"], world, res["e2e_ms"]), "unit": "TFLOP/s",
                            "h2d_bytes_per_step": res["h2d_bytes"], "d2h_bytes_per_step": res["d2h_bytes"],
                            "ms_per_step": res["e2e_ms"], "pipeline": res.get("e2e_pipeline")}
+        if "mask" in res:
+            m = dict(res["mask"])
+            m["mask_to_lists_roofline"] = {"bound": "hbm", "achieved": m.pop("mask_to_lists_gbs"),
+                                           "peak": pk["hbm_gbs"], "unit": "GB/s"}
+            m["mask_to_lists_roofline"]["frac"] = m["mask_to_lists_roofline"]["achieved"] / pk["hbm_gbs"]
+            line["mask_input"] = m
         if res["cpu"] is not None:
             line["cpu_baseline"] = res["cpu"]
         print(json.dumps(line), flush=True)

@@ -24,7 +24,7 @@ STATUS = {0: "BSA_OK", 1: "BSA_ERR_INVALID_ARG", 2: "BSA_ERR_UNSUPPORTED", 3: "B
 # Every symbol include/bsa.h declares.
 EXPORTS = ["bsa_tpd_budget", "bsa_score_workspace_bytes", "stem_score", "stem_select", "bsa_prefill",
            "bsa_prefill_paged", "bsa_last_error", "bsa_check_device_error", "stem_score_noalloc",
-           "bsa_selftest_wait_timeout"]
+           "bsa_selftest_wait_timeout", "bsa_mask_workspace_bytes", "bsa_mask_to_lists", "bsa_prefill_mask"]
 
 
 class BsaError(RuntimeError):
@@ -58,11 +58,15 @@ def lib():
     L.bsa_prefill.argtypes = [T, T, T, T, i32, i32, i32, i32, i32, i32, P, i32, P, i64, f32, P, P]
     L.bsa_prefill_paged.argtypes = [T, T, P, P, i32, T, T, i32, i32, P, i32, i32, i32, i32, i32, P, i32, P, i64,
                                     f32, P, P]
+    L.bsa_mask_workspace_bytes.argtypes = [i32, i32, i32]
+    L.bsa_mask_workspace_bytes.restype = ctypes.c_size_t
+    L.bsa_mask_to_lists.argtypes = [P, i64, i32, i32, i32, P, P, i64, P]
+    L.bsa_prefill_mask.argtypes = [T, T, T, T, i32, i32, i32, i32, i32, i32, P, i64, f32, P, P, ctypes.c_size_t, P]
     L.bsa_last_error.restype = ctypes.c_char_p
     L.bsa_check_device_error.argtypes = [P]
     L.bsa_selftest_wait_timeout.argtypes = [ctypes.c_uint64, P]
     for name in ["stem_score", "stem_score_noalloc", "stem_select", "bsa_prefill", "bsa_prefill_paged", "bsa_check_device_error",
-                 "bsa_selftest_wait_timeout"]:
+                 "bsa_selftest_wait_timeout", "bsa_mask_to_lists", "bsa_prefill_mask"]:
         getattr(L, name).restype = ctypes.c_int
     _lib = L
     return L
@@ -185,6 +189,65 @@ def bsa_prefill(q, k, v, block: int, row_ptr, col_idx, softmax_scale: float = 0.
     st = lib().bsa_prefill(tensor_arg(q, q_scale), tensor_arg(k, k_scale), tensor_arg(v, v_scale), tensor_arg(out),
                            B, N, Hq, Hkv, d, block, _ptr(row_ptr), row_ptr.shape[-1], _ptr(col_idx),
                            col_idx.shape[-1], float(softmax_scale), _ptr(lse), _stream(q))
+    _check(st)
+    return (out, lse) if return_lse else out
+
+
+def block_mask_buffer(B: int, Hq: int, nb: int, device=None, dtype=torch.uint8) -> torch.Tensor:
+    """A zeroed [B, Hq, nb, nb] block mask whose rows start every multiple of 16 bytes, as
+    bsa_prefill_mask needs (a view into a [B, Hq, nb, 16 * ceil(nb / 16)] buffer)."""
+    ms = 16 * ((nb + 15) // 16)
+    return torch.zeros(B, Hq, nb, ms, dtype=dtype, device=device)[..., :nb]
+
+
+def _mask_arg(block_mask: torch.Tensor, B: int, Hq: int, nb: int):
+    """(pointer, row stride) of a [B, Hq, nb, >= nb] uint8 / bool mask with unit last stride."""
+    if block_mask.dtype == torch.bool:
+        block_mask = block_mask.view(torch.uint8)
+    if block_mask.dtype != torch.uint8:
+        raise TypeError("block_mask must be uint8 or bool")
+    if block_mask.dim() != 4 or tuple(block_mask.shape[:3]) != (B, Hq, nb) or block_mask.shape[3] < nb:
+        raise ValueError(f"block_mask must be [B={B}, Hq={Hq}, nb={nb}, >= nb]")
+    ms = block_mask.stride(2)
+    if block_mask.stride(3) != 1 or block_mask.stride(1) != nb * ms or block_mask.stride(0) != Hq * nb * ms:
+        raise ValueError("block_mask must be dense apart from row padding (see block_mask_buffer)")
+    return ctypes.c_void_p(block_mask.data_ptr()), ms
+
+
+def bsa_mask_workspace_bytes(B: int, Hq: int, nb: int) -> int:
+    return int(lib().bsa_mask_workspace_bytes(B, Hq, nb))
+
+
+def bsa_mask_to_lists(block_mask: torch.Tensor, row_ptr=None, col_idx=None):
+    """Per-head lists of a block mask: (row_ptr [B, Hq, nb+1], col_idx [B, Hq, nb(nb+1)/2]) int32."""
+    B, Hq, nb = block_mask.shape[:3]
+    ptr, ms = _mask_arg(block_mask, B, Hq, nb)
+    cap = nb * (nb + 1) // 2
+    if row_ptr is None:
+        row_ptr = torch.empty(B, Hq, nb + 1, dtype=torch.int32, device=block_mask.device)
+    if col_idx is None:
+        col_idx = torch.empty(B, Hq, cap, dtype=torch.int32, device=block_mask.device)
+    _check(lib().bsa_mask_to_lists(ptr, ms, B, Hq, nb, _ptr(row_ptr), _ptr(col_idx), col_idx.shape[-1],
+                                   _stream(block_mask)))
+    return row_ptr, col_idx
+
+
+def bsa_prefill_mask(q, k, v, block: int, block_mask, softmax_scale: float = 0.0, out=None, lse=None,
+                     return_lse: bool = False, q_scale=1.0, k_scale=1.0, v_scale=1.0, workspace=None):
+    """Block-sparse causal prefill from a block mask [B, Hq, nb, >= nb] (uint8 / bool)."""
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    nb = (N + block - 1) // block
+    ptr, ms = _mask_arg(block_mask, B, Hq, nb)
+    if out is None:
+        out = torch.empty(B, N, Hq, d, dtype=torch.bfloat16, device=q.device)
+    if return_lse and lse is None:
+        lse = torch.empty(B, Hq, N, dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(max(bsa_mask_workspace_bytes(B, Hq, nb), 1), dtype=torch.uint8, device=q.device)
+    st = lib().bsa_prefill_mask(tensor_arg(q, q_scale), tensor_arg(k, k_scale), tensor_arg(v, v_scale), tensor_arg(out),
+                                B, N, Hq, Hkv, d, block, ptr, ms, float(softmax_scale), _ptr(lse),
+                                _ptr(workspace), workspace.numel(), _stream(q))
     _check(st)
     return (out, lse) if return_lse else out
 

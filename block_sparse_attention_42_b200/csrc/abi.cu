@@ -178,6 +178,90 @@ bsa_status_t attn_common_checks(const bsa_tensor_t& q, const bsa_tensor_t& k, co
     return BSA_OK;
 }
 
+
+bsa_status_t prefill_checks(const bsa_tensor_t& q, const bsa_tensor_t& k, const bsa_tensor_t& v,
+                            const bsa_tensor_t& out, int32_t B, int32_t N, int32_t Hq, int32_t Hkv, int32_t d,
+                            int32_t block, const int32_t* row_ptr, const int32_t* col_idx, int64_t max_k) {
+    bsa_status_t st;
+    if ((st = check_tensor(q, "q", B > 1)) || (st = check_tensor(k, "k", B > 1)) || (st = check_tensor(v, "v", B > 1)) ||
+        (st = check_tensor(out, "out", B > 1)))
+        return st;
+    if ((st = attn_common_checks(q, k, v, out, Hq, Hkv, d, block, row_ptr, col_idx, max_k))) return st;
+    if (B < 1 || B > kMaxBatch || N < 1) return fail(BSA_ERR_INVALID_ARG, "bad B=%d / N=%d", B, N);
+    const int nb = (N + block - 1) / block;
+    if (nb > kMaxBlocks) return fail(BSA_ERR_UNSUPPORTED, "at most %d blocks per sequence", kMaxBlocks);
+    if (static_cast<int64_t>(Hkv) * nb * (Hq / Hkv) > 0x7FFFFFFFll) return fail(BSA_ERR_UNSUPPORTED, "grid too large");
+    return BSA_OK;
+}
+
+bsa_status_t prefill_launch(const bsa_tensor_t& q, const bsa_tensor_t& k, const bsa_tensor_t& v,
+                            const bsa_tensor_t& out, int32_t B, int32_t N, int32_t Hq, int32_t Hkv, int32_t d,
+                            int32_t block, const int32_t* row_ptr, int32_t row_ptr_stride, int32_t row_ptr_hstride,
+                            int32_t allow_empty, const int32_t* col_idx, int64_t max_k, float softmax_scale,
+                            float* lse, cudaStream_t stream) {
+    bsa_status_t st;
+    const int nb = (N + block - 1) / block;
+    bsa_status_t est;
+    unsigned* err = device_error_word(&est);
+    if (!err) return est;
+    const int eb = elt_bytes(q.dtype);
+    CUtensorMap tq, tk, tv;
+    if ((st = make_map(&tq, q.ptr, eb, d, N, Hq, B, q.stride_t, q.stride_h, B > 1 ? q.stride_b : q.stride_t * N, 128, "q")) ||
+        (st = make_map(&tk, k.ptr, eb, d, N, Hkv, B, k.stride_t, k.stride_h, B > 1 ? k.stride_b : k.stride_t * N, block, "k")) ||
+        (st = make_map(&tv, v.ptr, eb, d, N, Hkv, B, v.stride_t, v.stride_h, B > 1 ? v.stride_b : v.stride_t * N, block, "v")))
+        return st;
+    AttnArgs a;
+    std::memset(&a, 0, sizeof a);
+    a.B = B;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.d = d;
+    a.block = block;
+    a.nb_max = nb;
+    a.N = N;
+    a.cu_seqlens = nullptr;
+    for (int b = 0; b < B; ++b) a.seqlen[b] = N;
+    a.row_ptr = row_ptr;
+    a.row_ptr_stride = row_ptr_stride;
+    a.row_ptr_hstride = row_ptr_hstride;
+    a.allow_empty = allow_empty;
+    a.col_idx = col_idx;
+    a.max_k = max_k;
+    const float tau = softmax_scale > 0.f ? softmax_scale : 1.f / std::sqrt(static_cast<float>(d));
+    const bool fp8 = q.dtype == BSA_FP8_E4M3;
+    a.scale_log2 = tau * 1.4426950408889634f * (fp8 ? q.scale * k.scale : 1.f);
+    a.out_scale = fp8 ? v.scale : 1.f;
+    a.out = out.ptr;
+    a.osb = out.stride_b;
+    a.ost = out.stride_t;
+    a.osh = out.stride_h;
+    a.lse = lse;
+    a.lse_stride = N;
+    a.err = err;
+    cudaError_t e = launch_attn(fp8, false, tq, tk, tv, a, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "bsa_prefill launch");
+    return BSA_OK;
+}
+
+
+// bsa_prefill_mask workspace: row_ptr [B*Hq][nb+1] | col_idx [B*Hq][nb(nb+1)/2].
+size_t mask_ws_bytes(int32_t B, int32_t Hq, int32_t nb) {
+    return align256(sizeof(int32_t) * size_t(B) * Hq * (nb + 1)) +
+           sizeof(int32_t) * size_t(B) * Hq * (size_t(nb) * (nb + 1) / 2);
+}
+
+bsa_status_t mask_checks(const uint8_t* mask, int64_t mask_stride, int32_t B, int32_t Hq, int32_t nb) {
+    if (!mask) return fail(BSA_ERR_INVALID_ARG, "block_mask is null");
+    if (B < 1 || B > kMaxBatch || Hq < 1) return fail(BSA_ERR_INVALID_ARG, "bad B=%d / Hq=%d", B, Hq);
+    if (nb < 1 || nb > kMaxBlocks) return fail(BSA_ERR_UNSUPPORTED, "nb must be in [1, %d]", kMaxBlocks);
+    if (mask_stride < nb || mask_stride % 16 != 0)
+        return fail(BSA_ERR_INVALID_ARG, "mask_stride (%lld) must be >= nb (%d) and a multiple of 16",
+                    static_cast<long long>(mask_stride), nb);
+    if (reinterpret_cast<uintptr_t>(mask) & 15u) return fail(BSA_ERR_INVALID_ARG, "block_mask must be 16-byte aligned");
+    if (static_cast<int64_t>(B) * Hq > 0x7FFFFFFFll) return fail(BSA_ERR_UNSUPPORTED, "grid too large");
+    return BSA_OK;
+}
+
 }  // namespace
 
 void set_last_error(const char* msg) { g_last_error = msg; }
@@ -336,53 +420,84 @@ bsa_status_t bsa_prefill(bsa_tensor_t q, bsa_tensor_t k, bsa_tensor_t v, bsa_ten
                          int32_t row_ptr_stride, const int32_t* col_idx, int64_t max_k, float softmax_scale,
                          float* lse, cudaStream_t stream) {
     bsa_status_t st;
-    if ((st = check_tensor(q, "q", B > 1)) || (st = check_tensor(k, "k", B > 1)) || (st = check_tensor(v, "v", B > 1)) ||
-        (st = check_tensor(out, "out", B > 1)))
-        return st;
-    if ((st = attn_common_checks(q, k, v, out, Hq, Hkv, d, block, row_ptr, col_idx, max_k))) return st;
-    if (B < 1 || B > kMaxBatch || N < 1) return fail(BSA_ERR_INVALID_ARG, "bad B=%d / N=%d", B, N);
+    if ((st = prefill_checks(q, k, v, out, B, N, Hq, Hkv, d, block, row_ptr, col_idx, max_k))) return st;
     const int nb = (N + block - 1) / block;
-    if (nb > kMaxBlocks) return fail(BSA_ERR_UNSUPPORTED, "at most %d blocks per sequence", kMaxBlocks);
     if (row_ptr_stride < nb + 1) return fail(BSA_ERR_INVALID_ARG, "row_ptr_stride must be >= nb + 1");
-    if (static_cast<int64_t>(Hkv) * nb * (Hq / Hkv) > 0x7FFFFFFFll) return fail(BSA_ERR_UNSUPPORTED, "grid too large");
-    bsa_status_t est;
-    unsigned* err = device_error_word(&est);
-    if (!err) return est;
-    const int eb = elt_bytes(q.dtype);
-    CUtensorMap tq, tk, tv;
-    if ((st = make_map(&tq, q.ptr, eb, d, N, Hq, B, q.stride_t, q.stride_h, B > 1 ? q.stride_b : q.stride_t * N, 128, "q")) ||
-        (st = make_map(&tk, k.ptr, eb, d, N, Hkv, B, k.stride_t, k.stride_h, B > 1 ? k.stride_b : k.stride_t * N, block, "k")) ||
-        (st = make_map(&tv, v.ptr, eb, d, N, Hkv, B, v.stride_t, v.stride_h, B > 1 ? v.stride_b : v.stride_t * N, block, "v")))
-        return st;
-    AttnArgs a;
-    std::memset(&a, 0, sizeof a);
-    a.B = B;
-    a.Hq = Hq;
-    a.Hkv = Hkv;
-    a.d = d;
-    a.block = block;
-    a.nb_max = nb;
-    a.N = N;
-    a.cu_seqlens = nullptr;
-    for (int b = 0; b < B; ++b) a.seqlen[b] = N;
-    a.row_ptr = row_ptr;
-    a.row_ptr_stride = row_ptr_stride;
-    a.col_idx = col_idx;
-    a.max_k = max_k;
-    const float tau = softmax_scale > 0.f ? softmax_scale : 1.f / std::sqrt(static_cast<float>(d));
-    const bool fp8 = q.dtype == BSA_FP8_E4M3;
-    a.scale_log2 = tau * 1.4426950408889634f * (fp8 ? q.scale * k.scale : 1.f);
-    a.out_scale = fp8 ? v.scale : 1.f;
-    a.out = out.ptr;
-    a.osb = out.stride_b;
-    a.ost = out.stride_t;
-    a.osh = out.stride_h;
-    a.lse = lse;
-    a.lse_stride = N;
-    a.err = err;
-    cudaError_t e = launch_attn(fp8, false, tq, tk, tv, a, stream);
-    if (e != cudaSuccess) return cuda_fail(e, "bsa_prefill launch");
+    return prefill_launch(q, k, v, out, B, N, Hq, Hkv, d, block, row_ptr, row_ptr_stride, 0, 0, col_idx, max_k,
+                          softmax_scale, lse, stream);
+}
+
+size_t bsa_mask_workspace_bytes(int32_t B, int32_t Hq, int32_t nb) {
+    if (B < 1 || Hq < 1 || nb < 1 || nb > kMaxBlocks) return 0;
+    return mask_ws_bytes(B, Hq, nb);
+}
+
+bsa_status_t bsa_mask_to_lists(const uint8_t* block_mask, int64_t mask_stride, int32_t B, int32_t Hq, int32_t nb,
+                               int32_t* row_ptr, int32_t* col_idx, int64_t max_k, cudaStream_t stream) {
+    bsa_status_t st;
+    if ((st = mask_checks(block_mask, mask_stride, B, Hq, nb))) return st;
+    if (!row_ptr || !col_idx) return fail(BSA_ERR_INVALID_ARG, "row_ptr/col_idx are null");
+    if (max_k < static_cast<int64_t>(nb) * (nb + 1) / 2)
+        return fail(BSA_ERR_INVALID_ARG, "max_k (%lld) < nb(nb+1)/2 = %lld", static_cast<long long>(max_k),
+                    static_cast<long long>(nb) * (nb + 1) / 2);
+    MaskListArgs m;
+    std::memset(&m, 0, sizeof m);
+    m.mask = block_mask;
+    m.mask_stride = mask_stride;
+    m.Hq = Hq;
+    m.nb = nb;
+    m.N = 0;  // no outputs: an empty row is just an empty list
+    m.block = 1;
+    m.d = 0;
+    m.row_ptr = row_ptr;
+    m.col_idx = col_idx;
+    m.cap = max_k;
+    cudaError_t e = launch_mask_lists(m, B, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "mask list launch");
     return BSA_OK;
+}
+
+bsa_status_t bsa_prefill_mask(bsa_tensor_t q, bsa_tensor_t k, bsa_tensor_t v, bsa_tensor_t out, int32_t B, int32_t N,
+                              int32_t Hq, int32_t Hkv, int32_t d, int32_t block, const uint8_t* block_mask,
+                              int64_t mask_stride, float softmax_scale, float* lse, void* ws, size_t ws_bytes,
+                              cudaStream_t stream) {
+    bsa_status_t st;
+    if (!ws) return fail(BSA_ERR_WORKSPACE, "workspace is null");
+    // (the list pointers are checked once they are carved out of the workspace)
+    const int nb = N > 0 && block > 0 ? (N + block - 1) / block : 0;
+    if ((st = prefill_checks(q, k, v, out, B, N, Hq, Hkv, d, block, static_cast<const int32_t*>(ws),
+                             static_cast<const int32_t*>(ws), 1)))
+        return st;
+    if ((st = mask_checks(block_mask, mask_stride, B, Hq, nb))) return st;
+    const size_t need = mask_ws_bytes(B, Hq, nb);
+    if (ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u))
+        return fail(BSA_ERR_WORKSPACE, "workspace must be >= %zu bytes and 256-byte aligned", need);
+    int32_t* row_ptr = static_cast<int32_t*>(ws);
+    int32_t* col_idx = reinterpret_cast<int32_t*>(static_cast<char*>(ws) +
+                                                  align256(sizeof(int32_t) * size_t(B) * Hq * (nb + 1)));
+    const int64_t cap = static_cast<int64_t>(nb) * (nb + 1) / 2;
+    MaskListArgs m;
+    std::memset(&m, 0, sizeof m);
+    m.mask = block_mask;
+    m.mask_stride = mask_stride;
+    m.Hq = Hq;
+    m.nb = nb;
+    m.N = N;
+    m.block = block;
+    m.d = d;
+    m.row_ptr = row_ptr;
+    m.col_idx = col_idx;
+    m.cap = cap;
+    m.out = out.ptr;
+    m.osb = out.stride_b;
+    m.ost = out.stride_t;
+    m.osh = out.stride_h;
+    m.lse = lse;
+    m.lse_stride = N;
+    cudaError_t e = launch_mask_lists(m, B, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "mask list launch");
+    return prefill_launch(q, k, v, out, B, N, Hq, Hkv, d, block, row_ptr, Hq * (nb + 1), nb + 1, 1, col_idx, cap,
+                          softmax_scale, lse, stream);
 }
 
 bsa_status_t bsa_prefill_paged(bsa_tensor_t q, bsa_tensor_t out, const int32_t* cu_seqlens, const int32_t* seqlens_host,

@@ -89,6 +89,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int bs = a.block;
     const int nb = (n_tok + bs - 1) / bs;
     if (i >= nb) return;
+    // A row with no kept block (allowed only where its output is written elsewhere): leave
+    // before any barrier or TMEM allocation.
+    if (a.allow_empty) {
+        const int32_t* rp0 =
+            a.row_ptr + static_cast<int64_t>(b) * a.row_ptr_stride + static_cast<int64_t>(h) * a.row_ptr_hstride;
+        if (rp0[i + 1] == rp0[i]) return;
+    }
     const int tok0 = PAGED ? a.cu_seqlens[b] : 0;  // packed row of token 0 of this sequence
 
     if (tid == 0) {
@@ -108,7 +115,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_relinquish();
     }
     // The list of this (b, h, i): validated once, before the loop.
-    const int32_t* rp = a.row_ptr + static_cast<int64_t>(b) * a.row_ptr_stride;
+    const int32_t* rp = a.row_ptr + static_cast<int64_t>(b) * a.row_ptr_stride + static_cast<int64_t>(h) * a.row_ptr_hstride;
     const int l_begin = rp[i];
     const int n_list = rp[i + 1] - l_begin;
     const int32_t* gl = a.col_idx + (static_cast<int64_t>(b) * a.Hq + h) * a.max_k + l_begin;

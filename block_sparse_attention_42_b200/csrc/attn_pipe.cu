@@ -115,9 +115,10 @@ __global__ void __launch_bounds__(kThreadsP, 1)
     const int bs = a.block;
     const int nb = (n_tok + bs - 1) / bs;
     if (i >= nb) return;
-    const int32_t* rp = a.row_ptr + static_cast<int64_t>(b) * a.row_ptr_stride;
+    const int32_t* rp = a.row_ptr + static_cast<int64_t>(b) * a.row_ptr_stride + static_cast<int64_t>(h) * a.row_ptr_hstride;
     const int l_begin = rp[i];
     const int n_list = rp[i + 1] - l_begin;
+    if (n_list == 0 && a.allow_empty) return;
     if (n_list < 1 || n_list > kMaxBlocks || l_begin < 0 || l_begin + static_cast<int64_t>(n_list) > a.max_k) {
         if (tid == 0) atomicOr(a.err, kDevErrInvalidList);
         return;

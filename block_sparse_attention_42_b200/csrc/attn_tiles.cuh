@@ -31,12 +31,13 @@ __device__ __forceinline__ Tile decode_tile(const AttnArgs& a, int t) {
     T.n_list = 0;
     T.l_begin = 0;
     if (T.valid) {
-        const int32_t* rp = a.row_ptr + static_cast<int64_t>(T.b) * a.row_ptr_stride;
+        const int32_t* rp = a.row_ptr + static_cast<int64_t>(T.b) * a.row_ptr_stride +
+                            static_cast<int64_t>(T.h) * a.row_ptr_hstride;
         T.l_begin = __ldg(rp + T.i);
         T.n_list = __ldg(rp + T.i + 1) - T.l_begin;
         if (T.n_list < 1 || T.n_list > kMaxBlocks || T.l_begin < 0 ||
             T.l_begin + static_cast<int64_t>(T.n_list) > a.max_k) {
-            T.n_list = 0;  // corrupt row pointer: the tile is skipped
+            T.n_list = 0;  // empty or corrupt row pointer: the tile is skipped
         }
     }
     return T;

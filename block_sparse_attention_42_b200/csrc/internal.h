@@ -57,7 +57,10 @@ struct AttnArgs {
     const int32_t* cu_seqlens;   // paged layout: device prefix offsets (nullptr for dense)
     int32_t seqlen[kMaxBatch];   // per-sequence lengths (dense: all N)
     const int32_t* row_ptr;
-    int row_ptr_stride;
+    int row_ptr_stride;          // entries between sequences
+    int row_ptr_hstride;         // entries between query heads (0: one row_ptr for all heads)
+    int allow_empty;             // 1: an empty list is a row with no kept block (its output
+                                 // is written elsewhere), not an error
     const int32_t* col_idx;
     int64_t max_k;
     const int32_t* page_table;   // paged only
@@ -83,6 +86,24 @@ cudaError_t launch_attention_ws4(bool fp8, bool paged, const CUtensorMap& tq, co
                                  const CUtensorMap& tv, const AttnArgs& a, cudaStream_t s);
 cudaError_t launch_attention_ws3(bool fp8, bool paged, const CUtensorMap& tq, const CUtensorMap& tk,
                                  const CUtensorMap& tv, const AttnArgs& a, cudaStream_t s);
+
+// Block mask -> per-head CSR lists (mask.cu).  mask [B, Hq, nb, mask_stride] uint8 (16-byte
+// aligned, mask_stride a multiple of 16 and >= nb); row_ptr [B*Hq][nb+1]; col_idx [B*Hq][cap]
+// with cap >= nb(nb+1)/2.  Rows that keep nothing get O = 0 (BF16 out, element strides) and
+// LSE = -inf (if lse is not null) for their query tokens.
+struct MaskListArgs {
+    const uint8_t* mask;
+    int64_t mask_stride;
+    int Hq, nb, N, block, d;
+    int32_t* row_ptr;
+    int32_t* col_idx;
+    int64_t cap;
+    void* out;
+    int64_t osb, ost, osh;
+    float* lse;
+    int64_t lse_stride;
+};
+cudaError_t launch_mask_lists(const MaskListArgs& m, int B, cudaStream_t s);
 
 // Sets the message bsa_last_error() returns on this thread.
 void set_last_error(const char* msg);

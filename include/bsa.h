@@ -121,6 +121,30 @@ bsa_status_t bsa_prefill(bsa_tensor_t q, bsa_tensor_t k, bsa_tensor_t v, bsa_ten
                          const int32_t* row_ptr, int32_t row_ptr_stride, const int32_t* col_idx,
                          int64_t max_k, float softmax_scale, float* lse, cudaStream_t stream);
 
+/* Block-mask input [cn486 page, §二.2.2 BSA算子优化: the sparse kernel receives the selection
+ * as a block mask and derives the kept-block list from it before its inner loop].
+ * block_mask (device, uint8) is [B, Hq, nb, mask_stride] with nb = ceil(N / block): row
+ * (b, h, i) keeps block j <= i iff block_mask[b][h][i][j] != 0; entries above the diagonal
+ * are ignored.  mask_stride >= nb and a multiple of 16; block_mask 16-byte aligned.
+ *
+ * bsa_mask_to_lists writes the per-head lists: row_ptr [B*Hq][nb+1] (offsets into the
+ * (b, h) row of col_idx) and col_idx [B*Hq][max_k], max_k >= nb(nb+1)/2, kept blocks in
+ * ascending order.  An empty row is an empty list.
+ *
+ * bsa_prefill_mask runs bsa_mask_to_lists into `ws` (bsa_mask_workspace_bytes(B, Hq, nb)
+ * bytes, 256-byte aligned) and then the bsa_prefill kernel on those lists; arguments and
+ * outputs otherwise as in bsa_prefill.  A query block whose mask row keeps nothing has
+ * out = 0 and lse = -inf for its tokens.  The workspace size returns 0 for invalid sizes. */
+size_t bsa_mask_workspace_bytes(int32_t B, int32_t Hq, int32_t nb);
+bsa_status_t bsa_mask_to_lists(const uint8_t* block_mask, int64_t mask_stride, int32_t B,
+                               int32_t Hq, int32_t nb, int32_t* row_ptr, int32_t* col_idx,
+                               int64_t max_k, cudaStream_t stream);
+bsa_status_t bsa_prefill_mask(bsa_tensor_t q, bsa_tensor_t k, bsa_tensor_t v, bsa_tensor_t out,
+                              int32_t B, int32_t N, int32_t Hq, int32_t Hkv, int32_t d,
+                              int32_t block, const uint8_t* block_mask, int64_t mask_stride,
+                              float softmax_scale, float* lse, void* ws, size_t ws_bytes,
+                              cudaStream_t stream);
+
 /* Paged-KV variant.  q and out are packed varlen [sum N_b, Hq, d] (stride_b unused);
  * cu_seqlens (device, B+1) gives each sequence's first token; seqlens_host (host, B) its
  * length.  k_cache/v_cache are page pools [num_pages, page_size, Hkv, d] described with

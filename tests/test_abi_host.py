@@ -53,6 +53,15 @@ def test_host_budget_rejects_bad_args(lib):
     assert lib.bsa_tpd_budget(8, 1.5, 0.5, None) == -1
 
 
+def test_mask_workspace_bytes(lib):
+    # row_ptr [B*Hq][nb+1] (256-byte aligned) then col_idx [B*Hq][nb(nb+1)/2], int32
+    for B, Hq, nb in [(1, 8, 8), (2, 64, 1024), (4, 32, 2048), (1, 1, 1)]:
+        rp = 4 * B * Hq * (nb + 1)
+        assert lib.bsa_mask_workspace_bytes(B, Hq, nb) == (rp + 255) // 256 * 256 + 4 * B * Hq * nb * (nb + 1) // 2
+    assert lib.bsa_mask_workspace_bytes(1, 8, 2049) == 0
+    assert lib.bsa_mask_workspace_bytes(0, 8, 8) == 0
+
+
 def _t(ptr=0x10000, dtype=0, st=1024, sh=128, sb=1 << 20, scale=1.0):
     from block_sparse_attention_42_b200.binding import BsaTensor
     return BsaTensor(ptr, dtype, scale, sb, st, sh)
@@ -96,6 +105,24 @@ def test_argument_errors_return_status(lib):
     sl = (ctypes.c_int32 * 1)(1024)
     assert lib.bsa_prefill_paged(_t(), _t(), P(1), sl, 1, _t(), _t(), 100, 32, P(1), 16, 8, 8, 128, 128, P(1), 9,
                                  P(1), 36, 0.0, None, None) == 2
+    # block-mask input: stride a multiple of 16 and >= nb, a 16-byte aligned mask, room for the
+    # lists; nb at most 2048
+    ws_need = lib.bsa_mask_workspace_bytes(1, 8, 8)
+    assert lib.bsa_prefill_mask(_t(), _t(), _t(), _t(), 1, 1024, 8, 8, 128, 128, P(0x60000), 10, 0.0, None, ws,
+                                1 << 30, None) == 1
+    assert lib.bsa_prefill_mask(_t(), _t(), _t(), _t(), 1, 1024, 8, 8, 128, 128, P(0x60000), 0, 0.0, None, ws,
+                                1 << 30, None) == 1
+    assert lib.bsa_prefill_mask(_t(), _t(), _t(), _t(), 1, 1024, 8, 8, 128, 128, P(0x60008), 16, 0.0, None, ws,
+                                1 << 30, None) == 1
+    assert lib.bsa_prefill_mask(_t(), _t(), _t(), _t(), 1, 1024, 8, 8, 128, 128, None, 16, 0.0, None, ws,
+                                1 << 30, None) == 1
+    assert lib.bsa_prefill_mask(_t(), _t(), _t(), _t(), 1, 1024, 8, 8, 128, 128, P(0x60000), 16, 0.0, None, ws,
+                                ws_need - 1, None) == 4
+    assert lib.bsa_prefill_mask(_t(), _t(), _t(), _t(), 1, 1024, 8, 8, 128, 128, P(0x60000), 16, 0.0, None, None,
+                                1 << 30, None) == 4
+    assert lib.bsa_mask_to_lists(P(0x60000), 16, 1, 8, 8, P(0x40000), P(0x50000), 35, None) == 1   # max_k < 36
+    assert lib.bsa_mask_to_lists(P(0x60000), 16, 1, 8, 8, None, P(0x50000), 36, None) == 1
+    assert lib.bsa_mask_to_lists(P(0x60000), 2064, 1, 8, 2049, P(0x40000), P(0x50000), 1 << 22, None) == 2
     # wait-timeout self-test: the limit must lie in [1 us, 1 s]
     assert lib.bsa_selftest_wait_timeout(ctypes.c_uint64(0), None) == 1
     assert lib.bsa_selftest_wait_timeout(ctypes.c_uint64(2_000_000_000), None) == 1
