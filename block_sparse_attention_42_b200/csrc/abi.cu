@@ -258,7 +258,8 @@ bsa_status_t mask_checks(const uint8_t* mask, int64_t mask_stride, int32_t B, in
         return fail(BSA_ERR_INVALID_ARG, "mask_stride (%lld) must be >= nb (%d) and a multiple of 16",
                     static_cast<long long>(mask_stride), nb);
     if (reinterpret_cast<uintptr_t>(mask) & 15u) return fail(BSA_ERR_INVALID_ARG, "block_mask must be 16-byte aligned");
-    if (static_cast<int64_t>(B) * Hq > 0x7FFFFFFFll) return fail(BSA_ERR_UNSUPPORTED, "grid too large");
+    // one warp per mask row, eight rows per CTA, grid.x < 2^31
+    if (static_cast<int64_t>(B) * Hq * nb > 8ll * 0x7FFFFFFFll) return fail(BSA_ERR_UNSUPPORTED, "grid too large");
     return BSA_OK;
 }
 

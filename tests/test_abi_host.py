@@ -123,6 +123,7 @@ def test_argument_errors_return_status(lib):
     assert lib.bsa_mask_to_lists(P(0x60000), 16, 1, 8, 8, P(0x40000), P(0x50000), 35, None) == 1   # max_k < 36
     assert lib.bsa_mask_to_lists(P(0x60000), 16, 1, 8, 8, None, P(0x50000), 36, None) == 1
     assert lib.bsa_mask_to_lists(P(0x60000), 2064, 1, 8, 2049, P(0x40000), P(0x50000), 1 << 22, None) == 2
+    assert lib.bsa_mask_to_lists(P(0x60000), 2048, 256, 65535, 2048, P(0x40000), P(0x50000), 1 << 22, None) == 2
     # wait-timeout self-test: the limit must lie in [1 us, 1 s]
     assert lib.bsa_selftest_wait_timeout(ctypes.c_uint64(0), None) == 1
     assert lib.bsa_selftest_wait_timeout(ctypes.c_uint64(2_000_000_000), None) == 1
