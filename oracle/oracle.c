@@ -295,7 +295,8 @@ static int int_cmp(const void* a, const void* b) {
 /* Keep list of query block i: the sink block 0 and the diagonal block i, plus the k_i - 2
  * best-scoring blocks among 1..i-1 (NaN scores count as -inf; equal scores prefer the
  * smaller j), returned in ascending order.  Row 0 keeps only block 0.  [P1 §3.2 selection
- * by the metric within the budget; spec reading: sink and diagonal always kept.] */
+ * by the metric within the budget.  Keeping the sink block 0 and the diagonal block in every
+ * row is a reading: the pages do not print the rule.] */
 void orc_select_row(const double* srow /* S[i][0..i] */, int32_t i, int32_t k_i, int32_t* out) {
     if (i == 0) {
         out[0] = 0;

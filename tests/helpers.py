@@ -7,7 +7,7 @@ import math
 import numpy as np
 import torch
 
-# Tolerances (also written in the design doc):
+# Tolerances:
 SCORE_REL = 1e-5          # scores: |gpu - oracle| <= 1e-5 * max(|oracle|, condition scale)
 BF16_MAX_ABS = 2e-2       # BF16 attention output: |g - o| <= 2e-2 + BF16_ULP_REL * |o|
 BF16_ULP_REL = 4 * 2.0 ** -9   # four BF16 half-ulps: output rounding + P rounding + accumulation
