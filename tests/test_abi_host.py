@@ -7,6 +7,7 @@ from pathlib import Path
 
 import numpy as np
 import pytest
+import torch
 
 ROOT = Path(__file__).resolve().parent.parent
 
@@ -128,3 +129,25 @@ def test_argument_errors_return_status(lib):
     assert lib.bsa_selftest_wait_timeout(ctypes.c_uint64(0), None) == 1
     assert lib.bsa_selftest_wait_timeout(ctypes.c_uint64(2_000_000_000), None) == 1
     assert lib.bsa_last_error().decode() != ""
+
+
+def test_block_mask_buffer_and_argument_checks():
+    """The binding's mask marshalling: padded rows, bool accepted, bad layouts refused (CPU tensors;
+    nothing is launched)."""
+    from block_sparse_attention_42_b200 import binding
+    for nb in (1, 15, 16, 17, 1000):
+        m = binding.block_mask_buffer(2, 3, nb)
+        assert m.shape == (2, 3, nb, nb) and m.dtype == torch.uint8
+        assert m.stride(2) % 16 == 0 and m.stride(2) >= nb and m.stride(3) == 1
+        ptr, ms = binding._mask_arg(m, 2, 3, nb)
+        assert ms == m.stride(2) and ptr.value == m.data_ptr()
+    mb = binding.block_mask_buffer(1, 2, 20, dtype=torch.bool)
+    assert binding._mask_arg(mb, 1, 2, 20)[1] == 32
+    with pytest.raises(TypeError):
+        binding._mask_arg(torch.zeros(1, 2, 20, 32, dtype=torch.int32), 1, 2, 20)
+    with pytest.raises(ValueError):
+        binding._mask_arg(torch.zeros(1, 2, 19, 32, dtype=torch.uint8), 1, 2, 20)      # wrong nb
+    with pytest.raises(ValueError):
+        binding._mask_arg(torch.zeros(1, 2, 20, 32, dtype=torch.uint8)[..., ::2], 1, 2, 20)  # strided columns
+    with pytest.raises(ValueError):
+        binding._mask_arg(torch.zeros(1, 20, 2, 32, dtype=torch.uint8).transpose(1, 2), 1, 2, 20)  # heads not outer
