@@ -217,6 +217,8 @@ def run_ours(args, rank, world, device):
         if record is not None:
             record[0].record(stream)
         bsa.stem_score(q, k, v, w.block, scores=scores, workspace=ws, **scale_kw)
+        if record is not None:
+            record[3].record(stream)
         bsa.stem_select(scores, [nb] * B, w.density, 0.5, row_ptr=row_ptr, col_idx=col_idx, max_k=kstar)
         if record is not None:
             record[1].record(stream)
@@ -231,7 +233,7 @@ def run_ours(args, rank, world, device):
     eff = effective_flop(row_ptr, col_idx, [N] * B, w.block, D)
 
     # Timed region: K steps, per-step events on the launching stream.
-    per = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    per = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(device)
@@ -246,11 +248,14 @@ def run_ours(args, rank, world, device):
     total_ms = ev[0].elapsed_time(ev[1])
     select_ms = [per[s][0].elapsed_time(per[s][1]) for s in range(args.steps)]
     attn_ms = [per[s][1].elapsed_time(per[s][2]) for s in range(args.steps)]
+    score_call_ms = [per[s][0].elapsed_time(per[s][3]) for s in range(args.steps)]
+    select_call_ms = [per[s][3].elapsed_time(per[s][1]) for s in range(args.steps)]
     max_ms = reduce_max(total_ms, world, device)
     bsa.bsa_check_device_error(device)
 
     res = dict(total_ms=max_ms, ms_per_step=max_ms / args.steps, eff_flop=eff,
                select_ms=statistics.median(select_ms), attn_ms=statistics.median(attn_ms),
+               score_call_ms=statistics.median(score_call_ms), select_call_ms=statistics.median(select_call_ms),
                attn_ms_mean=sum(attn_ms) / len(attn_ms), clocks=clk.summary(), w=w, N=N, B=B, Hq=Hq, Hkv=Hkv,
                D=D, nb=nb, kstar=kstar, fp8=fp8)
 
@@ -579,6 +584,19 @@ def main():
             line["e2e"] = {"value": whole_job_tflops(res["eff_flop"], world, res["e2e_ms"]), "unit": "TFLOP/s",
                            "h2d_bytes_per_step": res["h2d_bytes"], "d2h_bytes_per_step": res["d2h_bytes"],
                            "ms_per_step": res["e2e_ms"], "pipeline": res.get("e2e_pipeline")}
+        # The selection path's HBM rates.  stem_score = pool + score GEMM: its bytes are the
+        # pool's (Q, K, V read once), so the rate is a lower bound on the pool kernel's.
+        # stem_select = TPD budget + top-k: the causal scores read once, the lists written.
+        elt = 1 if fp8 else 2
+        n_tok = res["B"] * res["N"]
+        pool_bytes = n_tok * (res["Hq"] + 2 * res["Hkv"]) * res["D"] * elt
+        causal = res["B"] * res["nb"] * (res["nb"] + 1) // 2
+        sel_bytes = 4 * res["Hq"] * causal + 4 * res["Hq"] * res["B"] * res["kstar"]
+        line["select_path"] = {
+            "stem_score_ms": res["score_call_ms"], "stem_select_ms": res["select_call_ms"],
+            "pool_bytes": pool_bytes, "pool_gbs_lower_bound": pool_bytes / (res["score_call_ms"] * 1e-3) / 1e9,
+            "select_bytes": sel_bytes, "select_gbs": sel_bytes / (res["select_call_ms"] * 1e-3) / 1e9,
+            "hbm_peak_gbs": pk["hbm_gbs"]}
         if "mask" in res:
             m = dict(res["mask"])
             m["mask_to_lists_roofline"] = {"bound": "hbm", "achieved": m.pop("mask_to_lists_gbs"),
