@@ -16,6 +16,9 @@
  *                list; a skipped block contributes exactly nothing (all of its scores are
  *                -inf).  The paged variant reads K/V from a page pool through a page table.
  *                [same page, §二.2.2 BSA算子优化.]
+ *   bsa_mask_to_lists / bsa_prefill_mask
+ *                the same attention with the selection given as a uint8 block mask per
+ *                (sequence, query head), the form HPC-BSA takes it in [same page, §二.2.2].
  *
  * Conventions shared by every call:
  *   - All pointers except those marked "host" are device pointers on the current device.
@@ -129,12 +132,16 @@ bsa_status_t bsa_prefill(bsa_tensor_t q, bsa_tensor_t k, bsa_tensor_t v, bsa_ten
  *
  * bsa_mask_to_lists writes the per-head lists: row_ptr [B*Hq][nb+1] (offsets into the
  * (b, h) row of col_idx) and col_idx [B*Hq][max_k], max_k >= nb(nb+1)/2, kept blocks in
- * ascending order.  An empty row is an empty list.
+ * ascending order.  An empty row is an empty list.  Errors: a null, misaligned or
+ * badly strided mask, max_k < nb(nb+1)/2 or null lists -> BSA_ERR_INVALID_ARG; nb outside
+ * [1, 2048] or a row grid past the launch limit -> BSA_ERR_UNSUPPORTED; nothing launched.
  *
  * bsa_prefill_mask runs bsa_mask_to_lists into `ws` (bsa_mask_workspace_bytes(B, Hq, nb)
  * bytes, 256-byte aligned) and then the bsa_prefill kernel on those lists; arguments and
  * outputs otherwise as in bsa_prefill.  A query block whose mask row keeps nothing has
- * out = 0 and lse = -inf for its tokens.  The workspace size returns 0 for invalid sizes. */
+ * out = 0 and lse = -inf for its tokens.  A missing, misaligned (256 bytes) or short
+ * workspace -> BSA_ERR_WORKSPACE; the mask and tensor checks as above and in bsa_prefill.
+ * bsa_mask_workspace_bytes returns 0 for invalid sizes. */
 size_t bsa_mask_workspace_bytes(int32_t B, int32_t Hq, int32_t nb);
 bsa_status_t bsa_mask_to_lists(const uint8_t* block_mask, int64_t mask_stride, int32_t B,
                                int32_t Hq, int32_t nb, int32_t* row_ptr, int32_t* col_idx,
