@@ -24,7 +24,8 @@ STATUS = {0: "BSA_OK", 1: "BSA_ERR_INVALID_ARG", 2: "BSA_ERR_UNSUPPORTED", 3: "B
 # Every symbol include/bsa.h declares.
 EXPORTS = ["bsa_tpd_budget", "bsa_score_workspace_bytes", "stem_score", "stem_select", "bsa_prefill",
            "bsa_prefill_paged", "bsa_last_error", "bsa_check_device_error", "stem_score_noalloc",
-           "bsa_selftest_wait_timeout", "bsa_mask_workspace_bytes", "bsa_mask_to_lists", "bsa_prefill_mask"]
+           "bsa_selftest_wait_timeout", "bsa_mask_workspace_bytes", "bsa_mask_to_lists", "bsa_prefill_mask",
+           "bsa_validate_lists"]
 
 
 class BsaError(RuntimeError):
@@ -62,11 +63,12 @@ def lib():
     L.bsa_mask_workspace_bytes.restype = ctypes.c_size_t
     L.bsa_mask_to_lists.argtypes = [P, i64, i32, i32, i32, P, P, i64, P]
     L.bsa_prefill_mask.argtypes = [T, T, T, T, i32, i32, i32, i32, i32, i32, P, i64, f32, P, P, ctypes.c_size_t, P]
+    L.bsa_validate_lists.argtypes = [P, i64, i64, P, i64, i32, i32, P, i32, P]
     L.bsa_last_error.restype = ctypes.c_char_p
     L.bsa_check_device_error.argtypes = [P]
     L.bsa_selftest_wait_timeout.argtypes = [ctypes.c_uint64, P]
     for name in ["stem_score", "stem_score_noalloc", "stem_select", "bsa_prefill", "bsa_prefill_paged", "bsa_check_device_error",
-                 "bsa_selftest_wait_timeout", "bsa_mask_to_lists", "bsa_prefill_mask"]:
+                 "bsa_selftest_wait_timeout", "bsa_mask_to_lists", "bsa_prefill_mask", "bsa_validate_lists"]:
         getattr(L, name).restype = ctypes.c_int
     _lib = L
     return L
@@ -250,6 +252,24 @@ def bsa_prefill_mask(q, k, v, block: int, block_mask, softmax_scale: float = 0.0
                                 _ptr(workspace), workspace.numel(), _stream(q))
     _check(st)
     return (out, lse) if return_lse else out
+
+
+def bsa_validate_lists(row_ptr, col_idx, nb_per_seq, allow_empty: bool = False):
+    """Debug check of a list set: row_ptr [B, nbs+1] (one per sequence, as stem_select writes) or
+    [B, Hq, nb+1] (per head, as bsa_mask_to_lists writes); col_idx [B, Hq, max_k].  A violation
+    shows up in bsa_check_device_error (BSA_ERR_INVALID_LIST)."""
+    B, Hq, max_k = col_idx.shape
+    if row_ptr.dim() == 2:
+        rs, hs = row_ptr.stride(0), 0
+    elif row_ptr.dim() == 3:
+        rs, hs = row_ptr.stride(0), row_ptr.stride(1)
+    else:
+        raise ValueError("row_ptr must be [B, nbs+1] or [B, Hq, nb+1]")
+    if row_ptr.stride(-1) != 1:
+        raise ValueError("row_ptr rows must be contiguous")
+    nbp = torch.tensor([int(n) for n in nb_per_seq], dtype=torch.int32)
+    _check(lib().bsa_validate_lists(_ptr(row_ptr), rs, hs, _ptr(col_idx), max_k, B, Hq,
+                                    ctypes.c_void_p(nbp.data_ptr()), 1 if allow_empty else 0, _stream(col_idx)))
 
 
 def bsa_prefill_paged(q, cu_seqlens, seqlens, k_cache, v_cache, page_table, block: int, row_ptr, col_idx,

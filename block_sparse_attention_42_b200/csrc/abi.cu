@@ -458,6 +458,42 @@ bsa_status_t bsa_mask_to_lists(const uint8_t* block_mask, int64_t mask_stride, i
     return BSA_OK;
 }
 
+bsa_status_t bsa_validate_lists(const int32_t* row_ptr, int64_t row_ptr_stride, int64_t row_ptr_head_stride,
+                                const int32_t* col_idx, int64_t max_k, int32_t B, int32_t Hq,
+                                const int32_t* nb_per_seq, int32_t allow_empty, cudaStream_t stream) {
+    if (!row_ptr || !col_idx || !nb_per_seq) return fail(BSA_ERR_INVALID_ARG, "null pointer argument");
+    if (B < 1 || B > kMaxBatch) return fail(BSA_ERR_UNSUPPORTED, "B must be in [1, %d]", kMaxBatch);
+    if (Hq < 1) return fail(BSA_ERR_INVALID_ARG, "Hq must be positive");
+    if (max_k < 1) return fail(BSA_ERR_INVALID_ARG, "max_k must be positive");
+    ListCheckArgs c;
+    std::memset(&c, 0, sizeof c);
+    int nbmax = 0;
+    for (int b = 0; b < B; ++b) {
+        if (nb_per_seq[b] < 1 || nb_per_seq[b] > kMaxBlocks)
+            return fail(BSA_ERR_UNSUPPORTED, "nb_per_seq[%d] = %d outside [1, %d]", b, nb_per_seq[b], kMaxBlocks);
+        c.nb[b] = nb_per_seq[b];
+        nbmax = nb_per_seq[b] > nbmax ? nb_per_seq[b] : nbmax;
+    }
+    if (row_ptr_head_stride < 0 || (row_ptr_head_stride > 0 && row_ptr_head_stride < nbmax + 1) ||
+        row_ptr_stride < (row_ptr_head_stride > 0 ? row_ptr_head_stride * Hq : nbmax + 1))
+        return fail(BSA_ERR_INVALID_ARG, "row_ptr strides too small for %d blocks x %d heads", nbmax, Hq);
+    bsa_status_t est;
+    unsigned* err = device_error_word(&est);
+    if (!err) return est;
+    c.B = B;
+    c.Hq = Hq;
+    c.row_ptr = row_ptr;
+    c.rp_stride = row_ptr_stride;
+    c.rp_hstride = row_ptr_head_stride;
+    c.col_idx = col_idx;
+    c.max_k = max_k;
+    c.allow_empty = allow_empty ? 1 : 0;
+    c.err = err;
+    cudaError_t e = launch_validate_lists(c, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "list validation launch");
+    return BSA_OK;
+}
+
 bsa_status_t bsa_prefill_mask(bsa_tensor_t q, bsa_tensor_t k, bsa_tensor_t v, bsa_tensor_t out, int32_t B, int32_t N,
                               int32_t Hq, int32_t Hkv, int32_t d, int32_t block, const uint8_t* block_mask,
                               int64_t mask_stride, float softmax_scale, float* lse, void* ws, size_t ws_bytes,

@@ -105,6 +105,21 @@ struct MaskListArgs {
 };
 cudaError_t launch_mask_lists(const MaskListArgs& m, int B, cudaStream_t s);
 
+// Debug check of a CSR list set (validate.cu): records kDevErrInvalidList in *err on a
+// row_ptr out of order or past max_k, a row longer than i + 1 (or empty, unless allowed), or
+// entries not strictly ascending within [0, i].
+struct ListCheckArgs {
+    int B, Hq;
+    int32_t nb[kMaxBatch];
+    const int32_t* row_ptr;
+    int64_t rp_stride, rp_hstride;  // entries between sequences / query heads (0: shared)
+    const int32_t* col_idx;         // [B, Hq, max_k]
+    int64_t max_k;
+    int allow_empty;
+    unsigned* err;
+};
+cudaError_t launch_validate_lists(const ListCheckArgs& c, cudaStream_t s);
+
 // Sets the message bsa_last_error() returns on this thread.
 void set_last_error(const char* msg);
 cudaError_t launch_wait_timeout_selftest(unsigned* err, uint64_t limit_ns, cudaStream_t s);

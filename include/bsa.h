@@ -152,6 +152,21 @@ bsa_status_t bsa_prefill_mask(bsa_tensor_t q, bsa_tensor_t k, bsa_tensor_t v, bs
                               float softmax_scale, float* lse, void* ws, size_t ws_bytes,
                               cudaStream_t stream);
 
+/* Debug check of a kept-block list set, for lists that did not come from this library (or
+ * were edited).  row_ptr entries of (b, h) start at b * row_ptr_stride + h *
+ * row_ptr_head_stride (head stride 0: one row_ptr for all heads, as stem_select writes;
+ * nb + 1 with row_ptr_stride Hq * (nb + 1): bsa_mask_to_lists's layout); col_idx is
+ * [B, Hq, max_k]; nb_per_seq (host, B entries) gives each sequence's block count.  Checks
+ * every row (b, h, i): 0 <= row_ptr[i] <= row_ptr[i + 1] <= max_k, at most i + 1 entries
+ * (at least one unless allow_empty), entries strictly ascending within [0, i].  A violation
+ * is recorded in the device error word: bsa_check_device_error then returns
+ * BSA_ERR_INVALID_LIST.  Argument errors are returned synchronously (INVALID_ARG for null
+ * pointers, max_k < 1 or strides too small; UNSUPPORTED for B or nb out of range). */
+bsa_status_t bsa_validate_lists(const int32_t* row_ptr, int64_t row_ptr_stride,
+                                int64_t row_ptr_head_stride, const int32_t* col_idx,
+                                int64_t max_k, int32_t B, int32_t Hq, const int32_t* nb_per_seq,
+                                int32_t allow_empty, cudaStream_t stream);
+
 /* Paged-KV variant.  q and out are packed varlen [sum N_b, Hq, d] (stride_b unused);
  * cu_seqlens (device, B+1) gives each sequence's first token; seqlens_host (host, B) its
  * length.  k_cache/v_cache are page pools [num_pages, page_size, Hkv, d] described with

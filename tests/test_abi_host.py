@@ -125,6 +125,14 @@ def test_argument_errors_return_status(lib):
     assert lib.bsa_mask_to_lists(P(0x60000), 16, 1, 8, 8, None, P(0x50000), 36, None) == 1
     assert lib.bsa_mask_to_lists(P(0x60000), 2064, 1, 8, 2049, P(0x40000), P(0x50000), 1 << 22, None) == 2
     assert lib.bsa_mask_to_lists(P(0x60000), 2048, 256, 65535, 2048, P(0x40000), P(0x50000), 1 << 22, None) == 2
+    # list validation: null pointers, B / nb out of range, strides too small for nb
+    nb8 = (ctypes.c_int32 * 2)(8, 8)
+    assert lib.bsa_validate_lists(None, 9, 0, P(0x50000), 36, 1, 8, nb8, 0, None) == 1
+    assert lib.bsa_validate_lists(P(0x40000), 9, 0, P(0x50000), 36, 0, 8, nb8, 0, None) == 2
+    assert lib.bsa_validate_lists(P(0x40000), 9, 0, P(0x50000), 36, 1, 8, (ctypes.c_int32 * 1)(2049), 0, None) == 2
+    assert lib.bsa_validate_lists(P(0x40000), 8, 0, P(0x50000), 36, 1, 8, nb8, 0, None) == 1   # stride < nb + 1
+    assert lib.bsa_validate_lists(P(0x40000), 9 * 7, 9, P(0x50000), 36, 1, 8, nb8, 1, None) == 1  # < Hq * 9
+    assert lib.bsa_validate_lists(P(0x40000), 9, 0, P(0x50000), 0, 1, 8, nb8, 0, None) == 1   # max_k < 1
     # wait-timeout self-test: the limit must lie in [1 us, 1 s]
     assert lib.bsa_selftest_wait_timeout(ctypes.c_uint64(0), None) == 1
     assert lib.bsa_selftest_wait_timeout(ctypes.c_uint64(2_000_000_000), None) == 1
