@@ -458,3 +458,43 @@ def test_checks_catch_planted_mistakes(orc):
     for bad in [scores(lambda h: h % 2, True, qb), scores(lambda h: h // 2, False, qb),
                 scores(lambda h: h // 2, True, qb * bs)]:
         assert not np.allclose(bad[fin], ref[fin], rtol=1e-6)
+
+
+def test_mask_checks_catch_planted_mistakes():
+    """Slips a block-mask attention could make (the KV head's mask instead of the query head's,
+    the key's block as the mask row, no causal cut inside the diagonal block) planted in a
+    Python restatement fail the library-SDPA comparison that pins the oracle's mask function."""
+    rng = np.random.default_rng(14)
+    B, N, Hq, Hkv, D, bs = 1, 24, 4, 2, 4, 8
+    nb = N // bs
+    G = Hq // Hkv
+    q = rng.standard_normal((N, Hq, D)); k = rng.standard_normal((N, Hkv, D)); v = rng.standard_normal((N, Hkv, D))
+    mask = (rng.random((Hq, nb, nb)) < 0.5).astype(np.uint8)
+    for i in range(nb):
+        mask[:, i, 0] = 1                                    # every row keeps something
+    tau = 0.6
+
+    def attend(head_for_mask, row_of, causal):
+        out = np.zeros((Hq, N, D))
+        for h in range(Hq):
+            for t in range(N):
+                keys = [s for s in range(N) if mask[head_for_mask(h), row_of(t, s), s // bs]
+                        and (s <= t if causal else s // bs <= t // bs)]
+                lg = np.array([tau * q[t, h] @ k[s, h // G] for s in keys])
+                w = np.exp(lg - lg.max())
+                out[h, t] = (w[:, None] * v[keys, h // G]).sum(0) / w.sum()
+        return out
+
+    ref = np.zeros((Hq, N, D))
+    causal = torch.ones(N, N, dtype=torch.bool).tril()
+    for h in range(Hq):
+        tm = torch.from_numpy(np.kron(mask[h], np.ones((bs, bs), np.uint8)).astype(bool)) & causal
+        ref[h] = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(q[:, h]), torch.from_numpy(k[:, h // G]), torch.from_numpy(v[:, h // G]),
+            attn_mask=tm, scale=tau).numpy()
+    good = attend(lambda h: h, lambda t, s: t // bs, True)
+    np.testing.assert_allclose(good, ref, rtol=1e-12, atol=1e-12)
+    for bad in [attend(lambda h: h // G, lambda t, s: t // bs, True),      # KV head's mask
+                attend(lambda h: h, lambda t, s: s // bs, True),           # key block as the row
+                attend(lambda h: h, lambda t, s: t // bs, False)]:         # no causal cut
+        assert not np.allclose(bad, ref, rtol=1e-6, atol=1e-9)
