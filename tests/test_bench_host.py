@@ -48,3 +48,12 @@ def test_throughput_and_traffic_helpers(monkeypatch):
     assert bench.attn_traffic(False, 1, 32768, 64, 8, 128) is None
     monkeypatch.setenv("BSA_ATTN_VARIANT", "serial")
     assert bench.attn_traffic(True, 1, 32768, 64, 8, 128) is None
+
+
+def test_reference_arm_other_ranks_exit_without_work():
+    """Under torchrun only rank 0 runs and prints the reference line; the others exit 0 at once."""
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="", RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1", "--warmup", "0"],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    assert not [l for l in r.stdout.splitlines() if l.startswith("{")]
