@@ -69,9 +69,9 @@ def _load():
     lib.orc_select.argtypes = [P, ctypes.c_int, ctypes.c_int, P, ctypes.c_int, f64, f64, P, P, i64]
     lib.orc_select.restype = ctypes.c_int
     lib.orc_attention_rows.argtypes = [T, T, T, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-                                       ctypes.c_int, P, ctypes.c_int, P, i64, f64, P, i64, P, P]
+                                       ctypes.c_int, P, ctypes.c_int, P, i64, f64, P, i64, P, P, P]
     lib.orc_attention_rows_mask.argtypes = [T, T, T, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-                                            ctypes.c_int, P, i64, f64, P, i64, P, P]
+                                            ctypes.c_int, P, i64, f64, P, i64, P, P, P]
     lib.orc_effective_flop.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, P,
                                        ctypes.c_int, P, i64, ctypes.c_int]
     lib.orc_effective_flop.restype = f64
@@ -192,32 +192,39 @@ def select(S, nb_per_seq, density: float, decay: float = 0.5, maxK: int | None =
     return row_ptr, col_idx
 
 
-def attention_rows(q: View, k: View, v: View, N, Hq, Hkv, D, bs, row_ptr, col_idx, tau, rows):
-    """O and LSE (natural log) of the requested (b, h, t) query rows, fp64."""
+def attention_rows(q: View, k: View, v: View, N, Hq, Hkv, D, bs, row_ptr, col_idx, tau, rows,
+                   with_amp: bool = False):
+    """O and LSE (natural log) of the requested (b, h, t) query rows, fp64.  With with_amp,
+    also the softmax average of |v| per output element (see orc_attention_rows)."""
     row_ptr = _c(row_ptr, np.int32)
     col_idx = _c(col_idx, np.int32)
     rows = _c(rows, np.int64).reshape(-1, 3)
     n = rows.shape[0]
     out = np.empty((n, D), np.float64)
     lse = np.empty((n,), np.float64)
+    amp = np.empty((n, D), np.float64) if with_amp else None
     _load().orc_attention_rows(ctypes.byref(q.struct), ctypes.byref(k.struct), ctypes.byref(v.struct),
                                N, Hq, Hkv, D, bs, _ptr(row_ptr), row_ptr.shape[-1], _ptr(col_idx),
-                               col_idx.shape[-1], float(tau), _ptr(rows), n, _ptr(out), _ptr(lse))
-    return out, lse
+                               col_idx.shape[-1], float(tau), _ptr(rows), n, _ptr(out), _ptr(lse),
+                               None if amp is None else _ptr(amp))
+    return (out, lse, amp) if with_amp else (out, lse)
 
 
-def attention_rows_mask(q: View, k: View, v: View, N, Hq, Hkv, D, bs, mask, tau, rows):
+def attention_rows_mask(q: View, k: View, v: View, N, Hq, Hkv, D, bs, mask, tau, rows,
+                        with_amp: bool = False):
     """O and LSE of the requested (b, h, t) rows with the selection as a block mask
-    [B, Hq, nb, >= nb] (uint8; nonzero = kept), fp64.  Empty rows: O = 0, LSE = -inf."""
+    [B, Hq, nb, >= nb] (uint8; nonzero = kept), fp64.  Empty rows: O = 0, LSE = -inf.
+    With with_amp, also the softmax average of |v| per output element."""
     mask = np.ascontiguousarray(np.asarray(mask, dtype=np.uint8))
     rows = _c(rows, np.int64).reshape(-1, 3)
     n = rows.shape[0]
     out = np.empty((n, D), np.float64)
     lse = np.empty((n,), np.float64)
+    amp = np.empty((n, D), np.float64) if with_amp else None
     _load().orc_attention_rows_mask(ctypes.byref(q.struct), ctypes.byref(k.struct), ctypes.byref(v.struct),
                                     N, Hq, Hkv, D, bs, _ptr(mask), mask.shape[-1], float(tau), _ptr(rows), n,
-                                    _ptr(out), _ptr(lse))
-    return out, lse
+                                    _ptr(out), _ptr(lse), None if amp is None else _ptr(amp))
+    return (out, lse, amp) if with_amp else (out, lse)
 
 
 def effective_flop(N, Hq, D, bs, row_ptr, col_idx, b: int = 0) -> float:

@@ -31,7 +31,8 @@
  *                       reading of the pages: parity unpinned.
  *   orc_select          pinned: brute-force full sort; kept scores dominate dropped ones.
  *   orc_attention_rows  pinned: density 1 == library dense causal SDPA (fp64); skipped
- *                       blocks' contents are irrelevant; single-key closed form.
+ *                       blocks' contents are irrelevant; single-key closed form.  Its amp
+ *                       output == library SDPA with |V| as the values; single key: |v|.
  *   orc_attention_rows_mask  pinned: an all-ones mask == library dense causal SDPA; a
  *                       diagonal-only mask == library SDPA over the block's own keys; an
  *                       empty row gives 0 / -inf; entries above the diagonal are ignored.
@@ -355,11 +356,16 @@ int orc_select(const double* S /* [B][Hq][nbs][nbs] */, int B, int Hq, const int
  * keep list of (b, h, block(t))}; every other key has score -inf, so
  *     O = sum_{s in A(t)} softmax_s(tau * q_t . k_s) v_s,   lse = ln sum_{s in A(t)} e^{tau q.k}.
  * [P1 §二.2.2: a skipped block is mathematically a block of -inf scores, so softmax is exact.]
- * rows holds n_rows triples (b, h, t).  The mask is built explicitly per row. */
+ * rows holds n_rows triples (b, h, t).  The mask is built explicitly per row.
+ * amp (if not NULL) receives, per output element, the same softmax average of |v_s|:
+ *     amp = sum_{s in A(t)} softmax_s(tau * q_t . k_s) |v_s|,
+ * the magnitude a rounding of each weight by a relative eps can move O by at most eps * amp
+ * (used by the tests to bound the rounding of the weights to a 16-bit operand type). */
 void orc_attention_rows(const orc_tensor* q, const orc_tensor* k, const orc_tensor* v, int N,
                         int Hq, int Hkv, int D, int bs, const int32_t* row_ptr, int rp_stride,
                         const int32_t* col_idx, int64_t maxK, double tau, const int64_t* rows,
-                        int64_t n_rows, double* out /* [n_rows][D] */, double* lse /* [n_rows] */) {
+                        int64_t n_rows, double* out /* [n_rows][D] */, double* lse /* [n_rows] */,
+                        double* amp /* nullable [n_rows][D] */) {
     int G = Hq / Hkv;
 #pragma omp parallel
     {
@@ -394,14 +400,21 @@ void orc_attention_rows(const orc_tensor* q, const orc_tensor* k, const orc_tens
             }
             double z = 0.0;
             double* o = &out[r * D];
+            double* a = amp ? &amp[r * D] : NULL;
             for (int c = 0; c < D; ++c) o[c] = 0.0;
+            if (a)
+                for (int c = 0; c < D; ++c) a[c] = 0.0;
             for (int64_t s = 0; s < N; ++s) {
                 if (!allowed[s]) continue;
                 double w = exp(logit[s] - m);
                 z += w;
                 for (int c = 0; c < D; ++c) o[c] += w * load_elem(v, b, s, hk, c);
+                if (a)
+                    for (int c = 0; c < D; ++c) a[c] += w * fabs(load_elem(v, b, s, hk, c));
             }
             for (int c = 0; c < D; ++c) o[c] /= z;
+            if (a)
+                for (int c = 0; c < D; ++c) a[c] /= z;
             if (lse) lse[r] = m + log(z);
         }
         free(allowed);
@@ -415,11 +428,12 @@ void orc_attention_rows(const orc_tensor* q, const orc_tensor* k, const orc_tens
  * -inf scores].  mask is [B][Hq][nb][mask_stride] bytes; the allowed keys of query token t
  * (block i) of head h are A(t) = {s <= t : mask[b][h][i][block(s)] != 0}.  A row with A(t)
  * empty has no softmax; its output is taken as O = 0 and lse = -inf (the convention of
- * softmax over an empty set used by attention kernels).  The mask is read per key. */
+ * softmax over an empty set used by attention kernels).  The mask is read per key.
+ * amp as in orc_attention_rows (0 for an empty row). */
 void orc_attention_rows_mask(const orc_tensor* q, const orc_tensor* k, const orc_tensor* v, int N,
                              int Hq, int Hkv, int D, int bs, const uint8_t* mask, int64_t mask_stride,
                              double tau, const int64_t* rows, int64_t n_rows, double* out /* [n_rows][D] */,
-                             double* lse /* [n_rows] */) {
+                             double* lse /* [n_rows] */, double* amp /* nullable [n_rows][D] */) {
     int G = Hq / Hkv;
     int64_t nb = (N + bs - 1) / bs;
 #pragma omp parallel
@@ -443,7 +457,10 @@ void orc_attention_rows_mask(const orc_tensor* q, const orc_tensor* k, const orc
                 any = 1;
             }
             double* o = &out[r * D];
+            double* a = amp ? &amp[r * D] : NULL;
             for (int c = 0; c < D; ++c) o[c] = 0.0;
+            if (a)
+                for (int c = 0; c < D; ++c) a[c] = 0.0;
             if (!any) {
                 if (lse) lse[r] = -INFINITY;
                 continue;
@@ -454,8 +471,12 @@ void orc_attention_rows_mask(const orc_tensor* q, const orc_tensor* k, const orc
                 double w = exp(logit[s] - m);
                 z += w;
                 for (int c = 0; c < D; ++c) o[c] += w * load_elem(v, b, s, hk, c);
+                if (a)
+                    for (int c = 0; c < D; ++c) a[c] += w * fabs(load_elem(v, b, s, hk, c));
             }
             for (int c = 0; c < D; ++c) o[c] /= z;
+            if (a)
+                for (int c = 0; c < D; ++c) a[c] /= z;
             if (lse) lse[r] = m + log(z);
         }
         free(logit);

@@ -302,6 +302,39 @@ def test_skipped_blocks_are_irrelevant(orc):
     assert np.array_equal(base, pert)
 
 
+def test_amp_equals_library_sdpa_on_absolute_values(orc):
+    """The amp output (softmax average of |v| per output element) equals the library's SDPA
+    run with |V| as the values, under the same block-sparse causal mask; and it bounds |O|."""
+    w = inputs.Workload("pin", 1, 2, 1, 50, 8, 8, "fp32", 0.3, "stem", 95)
+    d = inputs.make_inputs(w)
+    q, k, v = d["q"].double(), d["k"].double(), d["v"].double()
+    B, N, Hq, Hkv, D, bs = 1, 50, 2, 1, 8, 8
+    nb = (N + bs - 1) // bs
+    S = np.random.default_rng(6).standard_normal((B, Hq, nb, nb))
+    rp, ci = orc.select(S, [nb], 0.3)
+    tau = 0.41
+    out, _, amp = orc.attention_rows(orc.view(q), orc.view(k), orc.view(v), N, Hq, Hkv, D, bs, rp, ci, tau,
+                                     _all_rows(B, Hq, N), with_amp=True)
+    for h in range(Hq):
+        mask = torch.zeros(N, N, dtype=torch.bool)
+        for i in range(nb):
+            for j in ci[0, h, rp[0, i]:rp[0, i + 1]]:
+                mask[i * bs:(i + 1) * bs, j * bs:(j + 1) * bs] = True
+        mask &= torch.ones(N, N, dtype=torch.bool).tril()
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            q[:, :, h], k[:, :, 0], v[:, :, 0].abs(), attn_mask=mask, scale=tau)[0]
+        np.testing.assert_allclose(amp[h * N:(h + 1) * N], ref.numpy(), rtol=1e-12, atol=1e-12)
+    assert np.all(np.abs(out) <= amp * (1 + 1e-12))
+    # the block-mask form gives the same amp for the same selection
+    mask = np.zeros((B, Hq, nb, nb), np.uint8)
+    for h in range(Hq):
+        for i in range(nb):
+            mask[0, h, i, ci[0, h, rp[0, i]:rp[0, i + 1]]] = 1
+    _, _, amp_m = orc.attention_rows_mask(orc.view(q), orc.view(k), orc.view(v), N, Hq, Hkv, D, bs, mask, tau,
+                                          _all_rows(B, Hq, N), with_amp=True)
+    np.testing.assert_allclose(amp_m, amp, rtol=1e-13, atol=0)
+
+
 def test_single_key_closed_form(orc):
     rng = np.random.default_rng(2)
     q = rng.standard_normal((1, 16, 1, 4)); k = rng.standard_normal((1, 16, 1, 4)); v = rng.standard_normal((1, 16, 1, 4))
@@ -310,6 +343,9 @@ def test_single_key_closed_form(orc):
                                   np.array([(0, 0, 0)], np.int64))
     assert np.array_equal(out[0], v[0, 0, 0])             # one allowed key: weight exactly 1
     assert lse[0] == pytest.approx(0.7 * float(q[0, 0, 0] @ k[0, 0, 0]), rel=1e-15)
+    _, _, amp = orc.attention_rows(orc.view(q), orc.view(k), orc.view(v), 16, 1, 1, 4, 8, rp, ci, 0.7,
+                                   np.array([(0, 0, 0)], np.int64), with_amp=True)
+    assert np.array_equal(amp[0], np.abs(v[0, 0, 0]))
 
 
 # ----------------------------------------------------------------------------- block-mask input
