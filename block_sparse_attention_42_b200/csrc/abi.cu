@@ -9,6 +9,8 @@
 #include <mutex>
 #include <string>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "../../include/bsa.h"
 #include "internal.h"
 
@@ -144,19 +146,25 @@ bsa_status_t make_map(CUtensorMap* m, const void* base, int eb, uint64_t d, uint
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// An NVTX range around one entry point, so a profiler's timeline shows each call of the C ABI
+// with the kernels it launched (header-only NVTX; a no-op unless a tool is attached).
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange&) = delete;
+    NvtxRange& operator=(const NvtxRange&) = delete;
+};
+
 // Attention kernel.  Default: ws3 (attn_ws3.cu: persistent, two pipelined CTAs per SM with a
 // TMA producer warp, an MMA warp and a softmax warpgroup; BF16 at d = 128 / block 128, whose
 // stages do not fit two CTAs per SM that way, runs ws2 with P in TMEM).  BSA_ATTN_VARIANT picks
-// another kernel: "serial" (attn.cu, one tile per CTA, no overlap inside a CTA), "pipe"
-// (attn_pipe.cu, one warpgroup that also issues), "ws4" (attn_ws4.cu, column-split softmax),
-// "ws2".  All compute the same result and the tests cross-check every one.
+// another kernel for cross-checks: "serial" (attn.cu, one tile per CTA, no overlap inside a
+// CTA) or "ws2".  All compute the same result and the tests cross-check every one.
 cudaError_t launch_attn(bool fp8, bool paged, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                         const AttnArgs& a, cudaStream_t s) {
     const char* v = std::getenv("BSA_ATTN_VARIANT");
     if (v && std::strcmp(v, "serial") == 0) return launch_attention(fp8, paged, tq, tk, tv, a, s);
     if (v && std::strcmp(v, "ws2") == 0) return launch_attention_ws2(fp8, paged, tq, tk, tv, a, s);
-    if (v && std::strcmp(v, "ws4") == 0) return launch_attention_ws4(fp8, paged, tq, tk, tv, a, s);
-    if (v && std::strcmp(v, "pipe") == 0) return launch_attention_pipe(fp8, paged, tq, tk, tv, a, s);
     return launch_attention_ws3(fp8, paged, tq, tk, tv, a, s);
 }
 
@@ -337,6 +345,7 @@ size_t bsa_score_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int32_t nb,
 bsa_status_t stem_score(bsa_tensor_t q, bsa_tensor_t k, bsa_tensor_t v, int32_t B, int32_t N, int32_t Hq,
                         int32_t Hkv, int32_t d, int32_t block, int32_t metric, float softmax_scale, float* scores,
                         int32_t nb_stride, void* ws, size_t ws_bytes, cudaStream_t stream) {
+    NvtxRange nvtx_range("stem_score");
     bsa_status_t st;
     if ((st = check_tensor(q, "q", B > 1)) || (st = check_tensor(k, "k", B > 1)) || (st = check_tensor(v, "v", B > 1)))
         return st;
@@ -393,6 +402,7 @@ bsa_status_t stem_score(bsa_tensor_t q, bsa_tensor_t k, bsa_tensor_t v, int32_t 
 bsa_status_t stem_select(const float* scores, int32_t B, int32_t Hq, const int32_t* nb_per_seq, int32_t nb_stride,
                          double density, double tpd_decay, int32_t* row_ptr, int32_t* col_idx, int64_t max_k,
                          cudaStream_t stream) {
+    NvtxRange nvtx_range("stem_select");
     if (!scores || !nb_per_seq || !row_ptr || !col_idx) return fail(BSA_ERR_INVALID_ARG, "null pointer argument");
     if (B < 1 || B > kMaxBatch) return fail(BSA_ERR_UNSUPPORTED, "B must be in [1, %d]", kMaxBatch);
     if (Hq < 1) return fail(BSA_ERR_INVALID_ARG, "Hq must be positive");
@@ -420,6 +430,7 @@ bsa_status_t bsa_prefill(bsa_tensor_t q, bsa_tensor_t k, bsa_tensor_t v, bsa_ten
                          int32_t Hq, int32_t Hkv, int32_t d, int32_t block, const int32_t* row_ptr,
                          int32_t row_ptr_stride, const int32_t* col_idx, int64_t max_k, float softmax_scale,
                          float* lse, cudaStream_t stream) {
+    NvtxRange nvtx_range("bsa_prefill");
     bsa_status_t st;
     if ((st = prefill_checks(q, k, v, out, B, N, Hq, Hkv, d, block, row_ptr, col_idx, max_k))) return st;
     const int nb = (N + block - 1) / block;
@@ -435,6 +446,7 @@ size_t bsa_mask_workspace_bytes(int32_t B, int32_t Hq, int32_t nb) {
 
 bsa_status_t bsa_mask_to_lists(const uint8_t* block_mask, int64_t mask_stride, int32_t B, int32_t Hq, int32_t nb,
                                int32_t* row_ptr, int32_t* col_idx, int64_t max_k, cudaStream_t stream) {
+    NvtxRange nvtx_range("bsa_mask_to_lists");
     bsa_status_t st;
     if ((st = mask_checks(block_mask, mask_stride, B, Hq, nb))) return st;
     if (!row_ptr || !col_idx) return fail(BSA_ERR_INVALID_ARG, "row_ptr/col_idx are null");
@@ -461,6 +473,7 @@ bsa_status_t bsa_mask_to_lists(const uint8_t* block_mask, int64_t mask_stride, i
 bsa_status_t bsa_validate_lists(const int32_t* row_ptr, int64_t row_ptr_stride, int64_t row_ptr_head_stride,
                                 const int32_t* col_idx, int64_t max_k, int32_t B, int32_t Hq,
                                 const int32_t* nb_per_seq, int32_t allow_empty, cudaStream_t stream) {
+    NvtxRange nvtx_range("bsa_validate_lists");
     if (!row_ptr || !col_idx || !nb_per_seq) return fail(BSA_ERR_INVALID_ARG, "null pointer argument");
     if (B < 1 || B > kMaxBatch) return fail(BSA_ERR_UNSUPPORTED, "B must be in [1, %d]", kMaxBatch);
     if (Hq < 1) return fail(BSA_ERR_INVALID_ARG, "Hq must be positive");
@@ -498,6 +511,7 @@ bsa_status_t bsa_prefill_mask(bsa_tensor_t q, bsa_tensor_t k, bsa_tensor_t v, bs
                               int32_t Hq, int32_t Hkv, int32_t d, int32_t block, const uint8_t* block_mask,
                               int64_t mask_stride, float softmax_scale, float* lse, void* ws, size_t ws_bytes,
                               cudaStream_t stream) {
+    NvtxRange nvtx_range("bsa_prefill_mask");
     bsa_status_t st;
     if (!ws) return fail(BSA_ERR_WORKSPACE, "workspace is null");
     // (the list pointers are checked once they are carved out of the workspace)
@@ -543,6 +557,7 @@ bsa_status_t bsa_prefill_paged(bsa_tensor_t q, bsa_tensor_t out, const int32_t* 
                                int32_t Hkv, int32_t d, int32_t block, const int32_t* row_ptr,
                                int32_t row_ptr_stride, const int32_t* col_idx, int64_t max_k, float softmax_scale,
                                float* lse, cudaStream_t stream) {
+    NvtxRange nvtx_range("bsa_prefill_paged");
     bsa_status_t st;
     if ((st = check_tensor(q, "q", false)) || (st = check_tensor(out, "out", false)) ||
         (st = check_tensor(k_cache, "k_cache", true)) || (st = check_tensor(v_cache, "v_cache", true)))

@@ -68,7 +68,7 @@ struct TileIter {
     int round, s, base, stride, total;
     bool active;
     Tile T;
-    __device__ void init(int s_, int base_, int stride_, int total_) {
+    __device__ __forceinline__ void init(int s_, int base_, int stride_, int total_) {
         s = s_;
         base = base_;
         stride = stride_;
@@ -76,7 +76,7 @@ struct TileIter {
         round = 0;
         active = true;
     }
-    __device__ void next(const AttnArgs& a) {
+    __device__ __forceinline__ void next(const AttnArgs& a) {
         while (true) {
             const int t = base + s + round * stride;
             ++round;

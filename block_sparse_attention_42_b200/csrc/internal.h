@@ -80,10 +80,6 @@ cudaError_t launch_attention_ws2(bool fp8, bool paged, const CUtensorMap& tq, co
 
 // As ws2, but P goes through shared memory so S(k+1) is computed while the softmax still works
 // on block k (attn_ws3.cu).  FP8, and BF16 shapes whose stages fit two CTAs per SM.
-cudaError_t launch_attention_pipe(bool fp8, bool paged, const CUtensorMap& tq, const CUtensorMap& tk,
-                                  const CUtensorMap& tv, const AttnArgs& a, cudaStream_t s);
-cudaError_t launch_attention_ws4(bool fp8, bool paged, const CUtensorMap& tq, const CUtensorMap& tk,
-                                 const CUtensorMap& tv, const AttnArgs& a, cudaStream_t s);
 cudaError_t launch_attention_ws3(bool fp8, bool paged, const CUtensorMap& tq, const CUtensorMap& tk,
                                  const CUtensorMap& tv, const AttnArgs& a, cudaStream_t s);
 

@@ -54,7 +54,10 @@ bsa_status_t stem_score_noalloc(bsa_tensor_t q, bsa_tensor_t k, bsa_tensor_t v, 
                                 int32_t Hkv, int32_t d, int32_t block, int32_t metric, float softmax_scale,
                                 float* scores, int32_t nb_stride, cudaStream_t stream) {
     using namespace bsa;
-    if (B <= 0 || N <= 0 || Hq <= 0 || Hkv <= 0 || d <= 0 || block <= 0)  // stem_score reports the bad size
+    // Sizes stem_score refuses for another reason (non-positive sizes, a head_dim, block or head
+    // ratio it does not take) go straight to it, so the caller gets the same error it gives.
+    if (B <= 0 || N <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || (d != 64 && d != 128) ||
+        (block != 64 && block != 128))
         return stem_score(q, k, v, B, N, Hq, Hkv, d, block, metric, softmax_scale, scores, nb_stride, nullptr, 0,
                           stream);
     const int nb = (N + block - 1) / block;
