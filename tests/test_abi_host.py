@@ -133,6 +133,16 @@ def test_argument_errors_return_status(lib):
     assert lib.bsa_validate_lists(P(0x40000), 8, 0, P(0x50000), 36, 1, 8, nb8, 0, None) == 1   # stride < nb + 1
     assert lib.bsa_validate_lists(P(0x40000), 9 * 7, 9, P(0x50000), 36, 1, 8, nb8, 1, None) == 1  # < Hq * 9
     assert lib.bsa_validate_lists(P(0x40000), 9, 0, P(0x50000), 0, 1, 8, nb8, 0, None) == 1   # max_k < 1
+    # allocation-free scoring: a size stem_score refuses for another reason gets stem_score's own
+    # error, even when the problem would also be too large for the fixed scratch
+    big = 1 << 20
+    assert lib.stem_score_noalloc(_t(), _t(), _t(), 1, big, 64, 8, 96, 128, 0, 0.0, sc, 8192, None) == 2
+    assert "head_dim" in lib.bsa_last_error().decode()
+    assert lib.stem_score_noalloc(_t(), _t(), _t(), 1, big, 64, 8, 128, 1, 0, 0.0, sc, 1 << 20, None) == 2
+    assert "block" in lib.bsa_last_error().decode()
+    assert lib.stem_score_noalloc(_t(), _t(), _t(), 1, big, 64, 12, 128, 128, 0, 0.0, sc, 8192, None) == 1
+    assert lib.stem_score_noalloc(_t(), _t(), _t(), 1, big, 64, 8, 128, 128, 0, 0.0, sc, 8192, None) == 2
+    assert "fixed scratch" in lib.bsa_last_error().decode()
     # wait-timeout self-test: the limit must lie in [1 us, 1 s]
     assert lib.bsa_selftest_wait_timeout(ctypes.c_uint64(0), None) == 1
     assert lib.bsa_selftest_wait_timeout(ctypes.c_uint64(2_000_000_000), None) == 1
