@@ -50,7 +50,7 @@ def test_fp8_128k_lists_scores_and_sampled_outputs(orc):
 
     # attention, sampled rows
     rows = H.sample_rows(B, Hq, N, w.block, n_heads=4, n_rand=40, seed=3)
-    ref, ref_lse = H.oracle_attention(orc, q, k, v, w.block, rp, ci, tau, rows, sq, sk, sv)
+    ref, ref_lse, _ = H.oracle_attention(orc, q, k, v, w.block, rp, ci, tau, rows, sq, sk, sv)
     got = H.gather_rows(out, rows)
     assert H.rel_l2(got, ref) <= H.FP8_REL_L2
     got_lse = np.array([lse[b, h, t].item() for b, h, t in rows])
@@ -89,9 +89,9 @@ def test_paged_varlen_full_size(orc):
     for b, n in enumerate(seqlens):
         qb = d["q"][cu[b]:cu[b + 1]].unsqueeze(0)
         rows = H.sample_rows(1, Hq, n, bs, n_heads=2, n_rand=16, seed=11 + b)
-        ref, ref_lse = H.oracle_attention(orc, qb, d["k_seq"][b].unsqueeze(0), d["v_seq"][b].unsqueeze(0), bs,
-                                          rp[b:b + 1], ci[b:b + 1], tau, rows)
+        ref, ref_lse, amp = H.oracle_attention(orc, qb, d["k_seq"][b].unsqueeze(0), d["v_seq"][b].unsqueeze(0),
+                                               bs, rp[b:b + 1], ci[b:b + 1], tau, rows)
         ob = out[cu[b]:cu[b + 1]].unsqueeze(0)
-        H.assert_bf16_close(H.gather_rows(ob, rows), ref)
+        H.assert_bf16_close(H.gather_rows(ob, rows), ref, amp)
         got_lse = np.array([lse[b, h, t].item() for _, h, t in rows])
         assert np.max(np.abs(got_lse - ref_lse)) <= H.LSE_ABS, b

@@ -18,7 +18,7 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
 
 
-@pytest.fixture(params=["ws3", "ws2", "ws4", "pipe", "serial"])
+@pytest.fixture(params=["ws3", "ws2", "serial"])
 def variant(request, monkeypatch):
     monkeypatch.setenv("BSA_ATTN_VARIANT", request.param)
     return request.param
@@ -47,7 +47,7 @@ def _random_mask(B, Hq, nb, p, seed, empty=(), full=()):
 def _oracle(orc, q, k, v, block, mask, rows, sq=1.0, sk=1.0, sv=1.0):
     B, N, Hq, d = q.shape
     return orc.attention_rows_mask(orc.view(q.cpu(), sq), orc.view(k.cpu(), sk), orc.view(v.cpu(), sv), N, Hq,
-                                   k.shape[2], d, block, mask.cpu().numpy(), H.default_tau(d), rows)
+                                   k.shape[2], d, block, mask.cpu().numpy(), H.default_tau(d), rows, with_amp=True)
 
 
 def _empty_rows(mask, N, block):
@@ -75,9 +75,9 @@ def test_mask_bf16_matches_oracle(orc, variant, name, w):
     out, lse = bsa.bsa_prefill_mask(q, k, v, w.block, mask, return_lse=True)
     bsa.bsa_check_device_error()
     rows = H.all_rows(B, Hq, N)
-    ref, ref_lse = _oracle(orc, q, k, v, w.block, mask, rows)
+    ref, ref_lse, amp = _oracle(orc, q, k, v, w.block, mask, rows)
     got = H.gather_rows(out, rows)
-    H.assert_bf16_close(got, ref)
+    H.assert_bf16_close(got, ref, amp)
     got_lse = lse.cpu().numpy().reshape(-1)            # [B, Hq, N] in (b, h, t) order, as rows
     empty = np.array([tuple(r) in _empty_rows(mask, N, w.block) for r in rows])
     assert empty.any() and not empty.all()
@@ -95,7 +95,7 @@ def test_mask_fp8_matches_oracle(orc, variant):
     out = bsa.bsa_prefill_mask(q, k, v, w.block, mask, q_scale=sq, k_scale=sk, v_scale=sv)
     bsa.bsa_check_device_error()
     rows = H.all_rows(B, Hq, N)
-    ref, _ = _oracle(orc, q, k, v, w.block, mask, rows, sq, sk, sv)
+    ref, _, _ = _oracle(orc, q, k, v, w.block, mask, rows, sq, sk, sv)
     got = H.gather_rows(out, rows)
     assert H.rel_l2(got, ref) <= H.FP8_REL_L2
     empty = np.array([tuple(r) in _empty_rows(mask, N, w.block) for r in rows])

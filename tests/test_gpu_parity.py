@@ -18,7 +18,7 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
 
 
-@pytest.fixture(params=["ws3", "ws2", "ws4", "pipe", "serial"])
+@pytest.fixture(params=["ws3", "ws2", "serial"])
 def variant(request, monkeypatch):
     """Attention kernel: every variant the library can run (ws3 is the default)."""
     monkeypatch.setenv("BSA_ATTN_VARIANT", request.param)
@@ -207,9 +207,9 @@ def test_attention_bf16_matches_oracle(orc, variant, name, w, N, storage, full):
     out, lse = bsa.bsa_prefill(q, k, v, w.block, rp, ci, return_lse=True)
     bsa.bsa_check_device_error()
     rows = H.all_rows(B, Hq, N) if full else H.sample_rows(B, Hq, N, w.block)
-    ref, ref_lse = H.oracle_attention(orc, q, k, v, w.block, rp, ci, H.default_tau(d), rows)
+    ref, ref_lse, amp = H.oracle_attention(orc, q, k, v, w.block, rp, ci, H.default_tau(d), rows)
     got = H.gather_rows(out, rows)
-    H.assert_bf16_close(got, ref)
+    H.assert_bf16_close(got, ref, amp)
     got_lse = np.array([lse[b, h, t].item() for b, h, t in rows]) if not full else \
         lse.permute(0, 1, 2).cpu().numpy().reshape(-1)
     assert np.max(np.abs(got_lse - ref_lse)) <= H.LSE_ABS
@@ -223,7 +223,7 @@ def test_attention_fp8_matches_oracle(orc, variant):
     out = bsa.bsa_prefill(q, k, v, w.block, rp, ci, q_scale=sq, k_scale=sk, v_scale=sv)
     bsa.bsa_check_device_error()
     rows = H.all_rows(B, Hq, N)
-    ref, _ = H.oracle_attention(orc, q, k, v, w.block, rp, ci, H.default_tau(d), rows, sq, sk, sv)
+    ref, _, _ = H.oracle_attention(orc, q, k, v, w.block, rp, ci, H.default_tau(d), rows, sq, sk, sv)
     got = H.gather_rows(out, rows)
     assert H.rel_l2(got, ref) <= H.FP8_REL_L2
 
@@ -235,10 +235,11 @@ def test_density_one_is_dense_causal(orc, variant):
     out = bsa.bsa_prefill(q, k, v, w.block, rp, ci)
     torch.cuda.synchronize()
     G = w.Hq // w.Hkv
-    ref = torch.nn.functional.scaled_dot_product_attention(
-        q.double().transpose(1, 2), k.double().repeat_interleave(G, 2).transpose(1, 2),
-        v.double().repeat_interleave(G, 2).transpose(1, 2), is_causal=True).transpose(1, 2)
-    H.assert_bf16_close(out.double().cpu().numpy(), ref.cpu().numpy())
+    qt, kt = q.double().transpose(1, 2), k.double().repeat_interleave(G, 2).transpose(1, 2)
+    vt = v.double().repeat_interleave(G, 2).transpose(1, 2)
+    ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, is_causal=True).transpose(1, 2)
+    amp = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt.abs(), is_causal=True).transpose(1, 2)
+    H.assert_bf16_close(out.double().cpu().numpy(), ref.cpu().numpy(), amp.cpu().numpy())
 
 
 def test_skipped_blocks_do_not_matter(variant):
@@ -324,9 +325,10 @@ def test_invalid_list_entry_is_flagged(variant):
     bsa.bsa_check_device_error()           # the word was cleared
 
 
-def test_variants_agree_at_full_size_sample(monkeypatch):
-    """The two attention kernels on the 8K GQA workload agree within twice the BF16 bound (each is
-    within the bound of the oracle; the per-row checks against the oracle are above)."""
+def test_variants_agree_at_full_size_sample(orc, monkeypatch):
+    """The serial kernel and the default kernel on the 8K GQA workload agree in rel-L2 over the
+    whole output, and on sampled rows within twice the BF16 bound (each is within the bound
+    of the oracle; the per-row checks against the oracle are above)."""
     w = inputs.gqa_8k()
     q, k, v, *_ = _inputs(w)
     rp, ci = _lists(q, k, v, w.block, w.density)
@@ -335,6 +337,8 @@ def test_variants_agree_at_full_size_sample(monkeypatch):
     monkeypatch.setenv("BSA_ATTN_VARIANT", "ws3")
     b = bsa.bsa_prefill(q, k, v, w.block, rp, ci)
     bsa.bsa_check_device_error()
-    a, b = a.double().cpu().numpy(), b.double().cpu().numpy()
-    assert np.all(np.abs(a - b) <= 2 * (H.BF16_MAX_ABS + H.BF16_ULP_REL * np.abs(a)))
-    assert H.rel_l2(b, a) <= H.BF16_REL_L2
+    assert H.rel_l2(b.double().cpu().numpy(), a.double().cpu().numpy()) <= H.BF16_REL_L2
+    rows = H.sample_rows(1, w.Hq, w.N, w.block, n_heads=4, n_rand=32, seed=9)
+    _, _, amp = H.oracle_attention(orc, q, k, v, w.block, rp, ci, H.default_tau(w.d), rows)
+    ga, gb = H.gather_rows(a, rows), H.gather_rows(b, rows)
+    assert np.all(np.abs(ga - gb) <= H.bf16_bound(ga, amp) + H.bf16_bound(gb, amp))
