@@ -13,6 +13,15 @@ Recipe (the pages run their operator benchmark on synthetic shapes; no dataset i
     by about 4 at scale 1/sqrt(d); every value row is scaled by exp(eta), eta ~ N(0, 1) per
     (token, kv head), so value amplitudes are log-normal and OAM and score-only selection
     differ.
+  * "blocky" distribution (only for the selection-quality record): keys carry a per-block
+    topic; each query block attends to a seeded set of key blocks whose values have a per-block
+    log-normal amplitude.  Per KV head, every key block j gets a seeded unit direction u_j and
+    every key of the block adds a * u_j; every query head h and query block i get a seeded set
+    J(h, i) = {0, i} plus up to 12 earlier blocks, and every query of block i adds a * u_j for j in
+    J(h, i), with a = sqrt(4 sqrt(d)) so a matched key lifts the logit by about 4 at scale
+    1/sqrt(d); every value row of block j is scaled by exp(eta_j), eta_j ~ N(0, 1) per (block, KV
+    head).  Attention then falls on whole blocks, more of them than a 25% budget keeps, with
+    different value amplitudes: the case the scoring metrics are meant to separate.
   * BF16 inputs are the fp32 draws rounded to nearest even; FP8 inputs are e4m3 codes of
     x / s with a per-tensor scale s = amax / 448 (torch's round-to-nearest-even cast).
   * Paged KV: 64-token pages, the pages of every sequence placed by a seeded permutation of
@@ -39,7 +48,7 @@ class Workload:
     block: int
     dtype: str                  # "fp32" | "bf16" | "fp8"
     density: float
-    dist: str                   # "normal" | "stem"
+    dist: str                   # "normal" | "stem" | "blocky"
     config_id: int
     seqlens: list = field(default_factory=list)  # varlen lengths (paged workloads)
     page_size: int = 0          # > 0: paged KV cache
@@ -75,13 +84,18 @@ def paged_varlen(density=0.25, seqlens=(16384, 32768, 65536, 131072)) -> Workloa
                     "stem", 4, seqlens=seqlens, page_size=64)
 
 
+def blocky_8k(density=0.25) -> Workload:
+    """The 8K GQA shape with block-structured attention (the selection-quality record only)."""
+    return Workload("blocky-8k", 1, 32, 8, 8192, 128, 128, "bf16", density, "blocky", 5)
+
+
 def fp8_32k(density=0.25) -> Workload:
     """The FP8 workload at 32K tokens: a profiling case that still exceeds L2 (Q is 268 MB)."""
     return Workload("fp8-32k", 1, 64, 8, 32768, 128, 128, "fp8", density, "stem", 3)
 
 
 WORKLOADS = {"tiny-1k": tiny, "gqa-8k": gqa_8k, "sweep-32k": sweep_32k, "fp8-128k": fp8_128k,
-             "paged-varlen": paged_varlen, "fp8-32k": fp8_32k}
+             "paged-varlen": paged_varlen, "fp8-32k": fp8_32k, "blocky-8k": blocky_8k}
 
 
 def _gen(device, seed):
@@ -110,6 +124,28 @@ def draw_fp32(w: Workload, B: int, N: int, device="cpu", seed_offset: int = 0):
         k[:, :64] += 2.0 * math.sqrt(d) * u
         eta = torch.randn(B, N, Hkv, 1, generator=_gen(dev, w.seed(5) + seed_offset), device=dev)
         v *= torch.exp(eta)
+    elif w.dist == "blocky":
+        nb = (N + w.block - 1) // w.block
+        gc = _gen(torch.device("cpu"), w.seed(3) + seed_offset)
+        u = torch.randn(B, Hkv, nb, d, generator=gc)
+        u = u / u.norm(dim=-1, keepdim=True)
+        amp = math.sqrt(4.0 * math.sqrt(d))
+        sel = torch.zeros(B, Hq, nb, nb)
+        for b in range(B):
+            for h in range(Hq):
+                for i in range(nb):
+                    sel[b, h, i, 0] = 1.0
+                    sel[b, h, i, i] = 1.0
+                    if i > 1:
+                        pick = torch.randperm(i - 1, generator=gc)[:12] + 1
+                        sel[b, h, i, pick] = 1.0
+        blk = torch.arange(N) // w.block
+        ku = u.permute(0, 2, 1, 3)[:, blk]                                        # [B, N, Hkv, d]
+        qtop = torch.einsum("bhij,bhjd->bhid", sel, u.repeat_interleave(G, dim=1))  # [B, Hq, nb, d]
+        k += (amp * ku).to(dev)
+        q += (amp * qtop.permute(0, 2, 1, 3)[:, blk]).to(dev)
+        eta = torch.randn(B, nb, Hkv, generator=gc)
+        v *= torch.exp(eta[:, blk]).unsqueeze(-1).to(dev)
     return q, k, v
 
 
