@@ -50,6 +50,9 @@ def parse():
                         "fastest at fp8-128k: 56.0 ms vs 57.3 / 62.3 for 2 / 4)")
     p.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
     p.add_argument("--no-mask", action="store_true", help="skip the block-mask input measurement")
+    p.add_argument("--no-sweeps", action="store_true",
+                   help="skip the density, length and paged-varlen sweeps of bsa_prefill")
+    p.add_argument("--sweep-reps", type=int, default=3, help="timed calls per sweep point")
     return p.parse_args()
 
 
@@ -182,6 +185,124 @@ def peaks():
         j = json.loads(p.read_text())
         return j, "measured"
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+# ----------------------------------------------------------------------------- sweeps
+
+SWEEP_DENSITIES = (0.10, 0.20, 0.25, 0.50, 0.80, 1.00)
+SWEEP_LENGTHS = (8192, 16384, 32768, 65536, 131072, 262144)
+
+
+def _time_calls(fn, reps, stream):
+    """Mean ms of `reps` back-to-back calls (CUDA events on the launching stream), after one
+    untimed call."""
+    fn()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def density_sweep(bsa, q, k, v, scores, block, seqlens, reps, stream, scale_kw):
+    """bsa_prefill over TPD lists at each density of SWEEP_DENSITIES, same inputs and scores:
+    ms, effective TFLOP/s and the ideal-line ratio ms / (dense ms x rho_eff), where rho_eff is
+    the ratio of effective FLOP to the density-1 (dense causal) FLOP."""
+    B, N, Hq, D = q.shape
+    nbp = [(n + block - 1) // block for n in seqlens]
+    out = torch.empty(B, N, Hq, D, dtype=torch.bfloat16, device=q.device)
+    pts = []
+    for rho in SWEEP_DENSITIES:
+        rp, ci = bsa.stem_select(scores, nbp, rho, 0.5)
+        ms = _time_calls(lambda: bsa.bsa_prefill(q, k, v, block, rp, ci, out=out, **scale_kw), reps, stream)
+        flop = effective_flop(rp, ci, seqlens, block, D)
+        pts.append({"density": rho, "ms": ms, "effective_flop": flop,
+                    "effective_tflops": flop / (ms * 1e-3) / 1e12})
+        del rp, ci
+    dense = pts[-1]
+    for pt in pts:
+        pt["rho_eff"] = pt["effective_flop"] / dense["effective_flop"]
+        pt["ideal_line_ratio"] = pt["ms"] / (dense["ms"] * pt["rho_eff"])
+    bsa.bsa_check_device_error(q.device)
+    return pts
+
+
+def run_sweeps(args, device, main):
+    """The pages' operator claims as measurements: latency linear in density (skip overhead),
+    stable throughput from 8K to 256K tokens at 75% sparsity, contiguous and paged KV, and the
+    paged varlen batch."""
+    import block_sparse_attention_42_b200 as bsa
+    from block_sparse_attention_42_b200 import inputs
+    stream = torch.cuda.current_stream(device)
+    reps = max(1, args.sweep_reps)
+    res = {"reps_per_point": reps}
+    with ClockSampler(device.index if device.index is not None else 0) as clk:
+        # (a) density sweep on the benchmark workload (same inputs and scores as the step) ...
+        res["density_sweep"] = {main["name"]: density_sweep(bsa, main["q"], main["k"], main["v"], main["scores"],
+                                                             main["block"], main["seqlens"], reps, stream,
+                                                             main["scale_kw"])}
+        # ... and on the BF16 32K workload
+        w = inputs.sweep_32k()
+        d = inputs.make_inputs(w, device=device)
+        S = bsa.stem_score(d["q"], d["k"], d["v"], w.block)
+        res["density_sweep"][w.name] = density_sweep(bsa, d["q"], d["k"], d["v"], S, w.block, [w.N] * w.B, reps,
+                                                      stream, {})
+        del d, S
+        # (b) length sweep: one sequence, 32 query / 8 KV heads, BF16, density 25%, the KV both
+        # contiguous and in 64-token pages placed by a seeded permutation
+        lens = []
+        for n in SWEEP_LENGTHS:
+            wl = inputs.Workload(f"single-{n // 1024}k", 1, 32, 8, n, 128, 128, "bf16", 0.25, "stem", 4,
+                                 seqlens=[n], page_size=64)
+            d = inputs.make_paged(wl, device=device)
+            q1, k1, v1 = d["q"].unsqueeze(0), d["k_seq"][0].unsqueeze(0), d["v_seq"][0].unsqueeze(0)
+            S = bsa.stem_score(q1, k1, v1, wl.block)
+            nb = S.shape[-1]
+            rp, ci = bsa.stem_select(S, [nb], wl.density)
+            del S
+            flop = effective_flop(rp, ci, [n], wl.block, wl.d)
+            out = torch.empty_like(q1, dtype=torch.bfloat16)
+            ms_c = _time_calls(lambda: bsa.bsa_prefill(q1, k1, v1, wl.block, rp, ci, out=out), reps, stream)
+            cu = d["cu_seqlens"].to(device)
+            outp = torch.empty_like(d["q"], dtype=torch.bfloat16)
+            ms_p = _time_calls(lambda: bsa.bsa_prefill_paged(d["q"], cu, [n], d["k_cache"], d["v_cache"],
+                                                             d["page_table"], wl.block, rp, ci, out=outp),
+                               reps, stream)
+            same = bool(torch.equal(out[0].view(torch.int16), outp.view(torch.int16)))
+            lens.append({"N": n, "effective_flop": flop, "contiguous_ms": ms_c,
+                         "contiguous_tflops": flop / (ms_c * 1e-3) / 1e12, "paged_ms": ms_p,
+                         "paged_tflops": flop / (ms_p * 1e-3) / 1e12, "paged_equals_contiguous": same})
+            del d, q1, k1, v1, rp, ci, out, outp
+        bsa.bsa_check_device_error(device)
+        res["length_sweep"] = {"config": "B1, 32/8 heads, d128, block 128, bf16, density 0.25 (75% sparsity)",
+                               "points": lens}
+        # (c) the paged varlen batch: 16K / 32K / 64K / 128K tokens, 32/8 heads, BF16 pages
+        wv = inputs.paged_varlen()
+        d = inputs.make_paged(wv, device=device)
+        seqlens, cu = d["seqlens"], d["cu_seqlens"]
+        nbp = [(n + wv.block - 1) // wv.block for n in seqlens]
+        nbs = max(nbp)
+        S = torch.full((len(seqlens), wv.Hq, nbs, nbs), float("nan"), device=device)
+        for b in range(len(seqlens)):
+            qb = d["q"][cu[b]:cu[b + 1]].unsqueeze(0)
+            bsa.stem_score(qb, d["k_seq"][b].unsqueeze(0), d["v_seq"][b].unsqueeze(0), wv.block,
+                           scores=S[b:b + 1], nb_stride=nbs)
+        rp, ci = bsa.stem_select(S, nbp, wv.density)
+        del S
+        cud = cu.to(device)
+        outp = torch.empty_like(d["q"], dtype=torch.bfloat16)
+        ms = _time_calls(lambda: bsa.bsa_prefill_paged(d["q"], cud, seqlens, d["k_cache"], d["v_cache"],
+                                                       d["page_table"], wv.block, rp, ci, out=outp), reps, stream)
+        flop = effective_flop(rp, ci, seqlens, wv.block, wv.d)
+        res["paged_varlen"] = {"workload": wv.name, "seqlens": seqlens, "Hq": wv.Hq, "Hkv": wv.Hkv, "dtype": "bf16",
+                               "density": wv.density, "ms": ms, "effective_flop": flop,
+                               "effective_tflops": flop / (ms * 1e-3) / 1e12}
+        bsa.bsa_check_device_error(device)
+        del d, outp, rp, ci
+    res["clocks"] = clk.summary()
+    return res
 
 
 # ----------------------------------------------------------------------------- our arm
@@ -386,7 +507,7 @@ def run_ours(args, rank, world, device):
         # the pipelined output equals the full-size call's
         for c in (0, NC - 1):
             assert torch.equal(hout[c], out[:, :, slq[c]].cpu()), "pipelined e2e output differs from the full call"
-        n_e2e = max(1, min(args.steps, 3))
+        n_e2e = max(1, args.steps)
         if world > 1:
             torch.distributed.barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -400,10 +521,15 @@ def run_ours(args, rank, world, device):
         e1.record(main)
         torch.cuda.synchronize(device)
         res["e2e_ms"] = reduce_max(e0.elapsed_time(e1) / n_e2e, world, device)
+        res["e2e_steps"] = n_e2e
         res["h2d_bytes"] = sum(x.numel() * x.element_size() for x in (q, k, v))
         res["d2h_bytes"] = out.numel() * out.element_size()
         res["e2e_pipeline"] = f"{NC} chunks ({G} KV-head groups x {F}), H2D / kernels / D2H on three streams"
         del hq, hk, hv, hout, dq, dk, dv, dout, g_scores, g_ws, g_rp, g_ci
+
+    if not args.no_sweeps and rank == 0:
+        res["sweeps"] = run_sweeps(args, device, dict(name=w.name, q=q, k=k, v=v, scores=scores, block=w.block,
+                                                      seqlens=[N] * B, scale_kw=scale_kw))
 
     res["cpu"] = None
     if not args.no_cpu and rank == 0:
@@ -419,16 +545,21 @@ def _oracle_sample_rows(w, N, Hq, n_rows, seed=0):
 
 
 def cpu_baseline(q, k, v, sq, sk, sv, row_ptr, col_idx, w, budget_s=12.0):
-    """The CPU oracle as it stands, on a bounded sample of the same workload: attention for
-    randomly sampled query rows (all host threads), effective TFLOP/s of those rows."""
+    """The CPU oracle as it stands, on the host cores:
+    - attention: randomly sampled query rows of the same workload and lists (all host threads,
+      then one thread), effective TFLOP/s of those rows;
+    - the select path exactly (pool + score + TPD budget + top-k over the whole workload), on all
+      host threads and on one."""
     import oracle
     oracle.build()
     qh, kh, vh = q.cpu(), k.cpu(), v.cpu()
     rp, ci = row_ptr.cpu().numpy(), col_idx.cpu().numpy()
     B, N, Hq, D = qh.shape
     Hkv = kh.shape[2]
+    nb = (N + w.block - 1) // w.block
     tau = 1.0 / math.sqrt(D)
     qv, kv, vv = oracle.view(qh, sq), oracle.view(kh, sk), oracle.view(vh, sv)
+    cores = len(os.sched_getaffinity(0))
 
     def row_flop(rows):
         f = 0.0
@@ -442,20 +573,41 @@ def cpu_baseline(q, k, v, sq, sk, sv, row_ptr, col_idx, w, budget_s=12.0):
                     f += hi - lo + 1
         return 4.0 * D * f
 
-    n, flop, secs, seed = 16, 0.0, 0.0, 0
-    while secs < budget_s:
-        rows = _oracle_sample_rows(w, N, Hq, n, seed)
+    def attention_sample(budget):
+        n, flop, secs, seed = 16, 0.0, 0.0, 0
+        while secs < budget:
+            rows = _oracle_sample_rows(w, N, Hq, n, seed)
+            t0 = time.perf_counter()
+            oracle.attention_rows(qv, kv, vv, N, Hq, Hkv, D, w.block, rp, ci, tau, rows)
+            secs += time.perf_counter() - t0
+            flop += row_flop(rows)
+            seed += 1
+            n = min(4096, n * 2)
+        return flop, secs
+
+    def select_path():
         t0 = time.perf_counter()
-        oracle.attention_rows(qv, kv, vv, N, Hq, Hkv, D, w.block, rp, ci, tau, rows)
-        dt = time.perf_counter() - t0
-        secs += dt
-        flop += row_flop(rows)
-        seed += 1
-        n = min(4096, n * 2)
-    cores = len(os.sched_getaffinity(0))
+        qb = oracle.pool_mean(qv, B, N, Hq, D, w.block)
+        kb = oracle.pool_mean(kv, B, N, Hkv, D, w.block)
+        vb = oracle.pool_vnorm(vv, B, N, Hkv, D, w.block)
+        S = oracle.score(qb, kb, vb, tau, 0)
+        oracle.select(S, [nb] * B, w.density, 0.5)
+        return time.perf_counter() - t0
+
+    oracle.set_threads(cores)
+    flop, secs = attention_sample(budget_s)
+    sel_s = select_path()
+    oracle.set_threads(1)
+    flop1, secs1 = attention_sample(budget_s / 3)
+    sel1_s = select_path()
+    oracle.set_threads(cores)
     return {"value": flop / secs / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
             "sample": f"fp64 oracle attention on {int(flop / 4 / D)} sampled (query, key) pairs of random "
-                      f"query rows of the same workload and lists, {secs:.1f} s on {cores} threads"}
+                      f"query rows of the same workload and lists, {secs:.1f} s on {cores} threads",
+            "one_core": {"value": flop1 / secs1 / 1e12, "unit": "TFLOP/s", "cores": 1,
+                         "sample": f"the same, {int(flop1 / 4 / D)} pairs, {secs1:.1f} s on one thread"},
+            "select_path": {"what": "pool + score + TPD budget + top-k over the whole workload (exact, not sampled)",
+                            "ms": 1e3 * sel_s, "cores": cores, "ms_one_core": 1e3 * sel1_s}}
 
 
 # ----------------------------------------------------------------------------- reference arm
@@ -583,7 +735,8 @@ def main():
         if "e2e_ms" in res:
             line["e2e"] = {"value": whole_job_tflops(res["eff_flop"], world, res["e2e_ms"]), "unit": "TFLOP/s",
                            "h2d_bytes_per_step": res["h2d_bytes"], "d2h_bytes_per_step": res["d2h_bytes"],
-                           "ms_per_step": res["e2e_ms"], "pipeline": res.get("e2e_pipeline")}
+                           "ms_per_step": res["e2e_ms"], "steps": res["e2e_steps"],
+                           "pipeline": res.get("e2e_pipeline")}
         # The selection path's HBM rates.  stem_score = pool + score GEMM: its bytes are the
         # pool's (Q, K, V read once), so the rate is a lower bound on the pool kernel's.
         # stem_select = TPD budget + top-k: the causal scores read once, the lists written.
@@ -597,6 +750,8 @@ def main():
             "pool_bytes": pool_bytes, "pool_gbs_lower_bound": pool_bytes / (res["score_call_ms"] * 1e-3) / 1e9,
             "select_bytes": sel_bytes, "select_gbs": sel_bytes / (res["select_call_ms"] * 1e-3) / 1e9,
             "hbm_peak_gbs": pk["hbm_gbs"]}
+        if "sweeps" in res:
+            line["sweeps"] = res["sweeps"]
         if "mask" in res:
             m = dict(res["mask"])
             m["mask_to_lists_roofline"] = {"bound": "hbm", "achieved": m.pop("mask_to_lists_gbs"),

@@ -75,6 +75,7 @@ def _load():
     lib.orc_effective_flop.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, P,
                                        ctypes.c_int, P, i64, ctypes.c_int]
     lib.orc_effective_flop.restype = f64
+    lib.orc_set_threads.argtypes = [ctypes.c_int]
     _lib = lib
     return lib
 
@@ -232,3 +233,9 @@ def effective_flop(N, Hq, D, bs, row_ptr, col_idx, b: int = 0) -> float:
     col_idx = _c(col_idx, np.int32)
     return _load().orc_effective_flop(N, Hq, D, bs, _ptr(row_ptr), row_ptr.shape[-1], _ptr(col_idx),
                                       col_idx.shape[-1], b)
+
+
+def set_threads(n: int) -> None:
+    """Host threads of the oracle's parallel loops from now on (timing only; results do not
+    depend on it)."""
+    _load().orc_set_threads(int(n))

@@ -42,6 +42,8 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <omp.h>
+
 #define ORC_F32 0
 #define ORC_BF16 1
 #define ORC_E4M3 2
@@ -505,3 +507,7 @@ double orc_effective_flop(int N, int Hq, int D, int bs, const int32_t* row_ptr, 
         }
     return 4.0 * D * pairs;
 }
+
+/* Number of host threads the parallel loops above use from now on (for timing the oracle on
+ * one core or on all of them; no effect on any result). */
+void orc_set_threads(int n) { omp_set_num_threads(n > 0 ? n : 1); }
