@@ -76,6 +76,7 @@ def _load():
                                        ctypes.c_int, P, i64, ctypes.c_int]
     lib.orc_effective_flop.restype = f64
     lib.orc_set_threads.argtypes = [ctypes.c_int]
+    lib.orc_group_mean.argtypes = [P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, P]
     _lib = lib
     return lib
 
@@ -149,6 +150,15 @@ def pool_vnorm(v: View, B, N, H, D, bs) -> np.ndarray:
     nb = (N + bs - 1) // bs
     out = np.empty((B, H, nb), np.float64)
     _load().orc_pool_vnorm(ctypes.byref(v.struct), B, N, H, D, bs, _ptr(out))
+    return out
+
+
+def group_mean(qbar, Hkv: int) -> np.ndarray:
+    """[B, Hq, nb, D] pooled queries -> [B, Hkv, nb, D] mean over each KV-head group's heads."""
+    qbar = _c(qbar, np.float64)
+    B, Hq, nb, D = qbar.shape
+    out = np.empty((B, Hkv, nb, D), np.float64)
+    _load().orc_group_mean(_ptr(qbar), B, Hq, Hkv, nb, D, _ptr(out))
     return out
 
 

@@ -26,6 +26,9 @@
  *   orc_pool_mean       pinned: brute-force mean of all token-pair logits == pooled score.
  *   orc_pool_vnorm      pinned: closed forms (constant rows, one-hot rows).
  *   orc_score           pinned: the pooled-GEMM equivalence above; -inf above the diagonal.
+ *   orc_group_mean      pinned: the group's score rows equal the mean of its heads' score rows
+ *                       (every metric is linear in the pooled query), and the brute-force mean
+ *                       over the group's heads and all token pairs; G = 1 is the identity.
  *   orc_tpd_budget      invariants pinned (sum, bounds, monotone keep ratio, density 1,
  *                       beta 0 uniform, hand-worked fixture).  The decay LAW itself is a
  *                       reading of the pages: parity unpinned.
@@ -187,6 +190,23 @@ void orc_score(const double* qbar /* [B][Hq][nb][D] */, const double* kbar /* [B
                     *dst = s;
                 }
         }
+}
+
+/* Group-shared selection (an extension: the pages select per query head and say nothing about
+ * grouped-query attention).  The query-side representation of KV-head group hk is the mean of
+ * its G = Hq / Hkv query heads' pooled Q:  gbar[b,hk,i,:] = (1/G) sum_{g<G} qbar[b, hk*G+g, i, :].
+ * orc_score on gbar (with Hq := Hkv) then gives the group's score rows. */
+void orc_group_mean(const double* qbar /* [B][Hq][nb][D] */, int B, int Hq, int Hkv, int nb, int D,
+                    double* gbar /* [B][Hkv][nb][D] */) {
+    int G = Hq / Hkv;
+    for (int b = 0; b < B; ++b)
+        for (int hk = 0; hk < Hkv; ++hk)
+            for (int i = 0; i < nb; ++i)
+                for (int c = 0; c < D; ++c) {
+                    double acc = 0.0;
+                    for (int g = 0; g < G; ++g) acc += qbar[(((int64_t)b * Hq + hk * G + g) * nb + i) * D + c];
+                    gbar[(((int64_t)b * Hkv + hk) * nb + i) * D + c] = acc / G;
+                }
 }
 
 /* ---------------------------------------------------------------- a3: TPD budget */

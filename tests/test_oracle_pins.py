@@ -96,6 +96,48 @@ def test_pooled_score_equals_token_pair_mean(orc, metric):
     np.testing.assert_allclose(S[fin], ref[fin], rtol=1e-12, atol=1e-12)
 
 
+@pytest.mark.parametrize("metric", [0, 1, 2])
+def test_group_score_is_mean_of_head_scores_and_of_token_pairs(orc, metric):
+    """Group-shared selection: the group's score row equals (a) the mean of its G heads' score
+    rows and (b) the brute-force mean over the group's heads and all token pairs of the block
+    pair (+ the value term).  A wrong head-to-group mapping or a sum for the mean fails both."""
+    rng = np.random.default_rng(11)
+    B, N, Hq, Hkv, D, bs = 2, 29, 6, 2, 8, 8   # G = 3, ragged tail
+    q = rng.standard_normal((B, N, Hq, D))
+    k = rng.standard_normal((B, N, Hkv, D))
+    v = rng.standard_normal((B, N, Hkv, D)) * np.exp(rng.standard_normal((B, N, Hkv, 1)))
+    tau = 1 / math.sqrt(D)
+    qb = orc.pool_mean(orc.view(q), B, N, Hq, D, bs)
+    kb = orc.pool_mean(orc.view(k), B, N, Hkv, D, bs)
+    vb = orc.pool_vnorm(orc.view(v), B, N, Hkv, D, bs)
+    Sg = orc.score(orc.group_mean(qb, Hkv), kb, vb, tau, metric)          # [B, Hkv, nb, nb]
+    Sh = orc.score(qb, kb, vb, tau, metric)                                # [B, Hq, nb, nb]
+    G = Hq // Hkv
+    nb = Sg.shape[-1]
+    fin = np.isfinite(Sg)
+    for hk in range(Hkv):
+        mean_rows = Sh[:, hk * G:(hk + 1) * G].mean(axis=1)
+        np.testing.assert_allclose(Sg[:, hk][fin[:, hk]], mean_rows[fin[:, hk]], rtol=1e-12, atol=1e-12)
+    # brute force over heads x token pairs
+    for b in range(B):
+        for hk in range(Hkv):
+            for i in range(nb):
+                for j in range(i + 1):
+                    tot, cnt = 0.0, 0
+                    for h in range(hk * G, (hk + 1) * G):
+                        for t in range(i * bs, min(N, (i + 1) * bs)):
+                            for s_ in range(j * bs, min(N, (j + 1) * bs)):
+                                tot += tau * float(np.dot(q[b, t, h], k[b, s_, hk]))
+                                cnt += 1
+                    val = tot / cnt
+                    amp = vb[b, hk, j]
+                    val = val + math.log(amp) if metric == 0 else (val * amp if metric == 2 else val)
+                    assert Sg[b, hk, i, j] == pytest.approx(val, rel=1e-11, abs=1e-11)
+    assert np.all(np.isneginf(Sg[..., np.triu_indices(nb, 1)[0], np.triu_indices(nb, 1)[1]]))
+    # G = 1: the group mean is the identity
+    assert np.array_equal(orc.group_mean(qb, Hq), qb)
+
+
 def test_vnorm_closed_forms(orc):
     D, bs = 16, 4
     v = np.zeros((1, 8, 2, D))
