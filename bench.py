@@ -53,6 +53,8 @@ def parse():
     p.add_argument("--no-sweeps", action="store_true",
                    help="skip the density, length and paged-varlen sweeps of bsa_prefill")
     p.add_argument("--sweep-reps", type=int, default=3, help="timed calls per sweep point")
+    p.add_argument("--no-group", action="store_true",
+                   help="skip the group-shared selection + GQA-packed attention measurement")
     return p.parse_args()
 
 
@@ -527,6 +529,35 @@ def run_ours(args, rank, world, device):
         res["e2e_pipeline"] = f"{NC} chunks ({G} KV-head groups x {F}), H2D / kernels / D2H on three streams"
         del hq, hk, hv, hout, dq, dk, dv, dout, g_scores, g_ws, g_rp, g_ci
 
+    # Group-shared selection (one list per KV-head group) and the GQA-packed attention kernel on
+    # the same inputs: the whole path timed like the step, plus the attention call alone.
+    if not args.no_group and rank == 0:
+        G = Hq // Hkv
+        g_scores = torch.empty(B, Hkv, nb, nb, dtype=torch.float32, device=device)
+        g_ws = torch.empty(bsa.bsa_score_group_workspace_bytes(B, Hq, Hkv, nb, D), dtype=torch.uint8, device=device)
+        g_rp = torch.empty(B, nb + 1, dtype=torch.int32, device=device)
+        g_ci = torch.empty(B, Hkv, kstar, dtype=torch.int32, device=device)
+        g_out = torch.empty_like(out)
+
+        def g_select():
+            bsa.stem_score_group(q, k, v, w.block, scores=g_scores, workspace=g_ws, **scale_kw)
+            bsa.stem_select(g_scores, [nb] * B, w.density, 0.5, row_ptr=g_rp, col_idx=g_ci, max_k=kstar)
+
+        def g_attn():
+            bsa.bsa_prefill_group(q, k, v, w.block, g_rp, g_ci, out=g_out, **scale_kw)
+
+        reps = max(3, min(args.steps, 10))
+        sel_ms = _time_calls(g_select, reps, stream)
+        attn_g_ms = _time_calls(g_attn, reps, stream)
+        bsa.bsa_check_device_error(device)
+        g_flop = G * effective_flop(g_rp, g_ci, [N] * B, w.block, D)
+        res["group"] = {"what": "stem_score_group + stem_select (one list per KV-head group) and bsa_prefill_group "
+                                "(two query heads per CTA, each kept K/V block loaded once for both)",
+                        "select_ms": sel_ms, "bsa_prefill_group_ms": attn_g_ms, "effective_flop": g_flop,
+                        "effective_tflops": g_flop / (attn_g_ms * 1e-3) / 1e12,
+                        "per_head_bsa_prefill_ms": res["attn_ms"], "reps": reps}
+        del g_scores, g_ws, g_rp, g_ci, g_out
+
     if not args.no_sweeps and rank == 0:
         res["sweeps"] = run_sweeps(args, device, dict(name=w.name, q=q, k=k, v=v, scores=scores, block=w.block,
                                                       seqlens=[N] * B, scale_kw=scale_kw))
@@ -752,6 +783,8 @@ def main():
             "hbm_peak_gbs": pk["hbm_gbs"]}
         if "sweeps" in res:
             line["sweeps"] = res["sweeps"]
+        if "group" in res:
+            line["group_shared"] = res["group"]
         if "mask" in res:
             m = dict(res["mask"])
             m["mask_to_lists_roofline"] = {"bound": "hbm", "achieved": m.pop("mask_to_lists_gbs"),

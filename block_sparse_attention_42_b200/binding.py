@@ -25,7 +25,7 @@ STATUS = {0: "BSA_OK", 1: "BSA_ERR_INVALID_ARG", 2: "BSA_ERR_UNSUPPORTED", 3: "B
 EXPORTS = ["bsa_tpd_budget", "bsa_score_workspace_bytes", "stem_score", "stem_select", "bsa_prefill",
            "bsa_prefill_paged", "bsa_last_error", "bsa_check_device_error", "stem_score_noalloc",
            "bsa_selftest_wait_timeout", "bsa_mask_workspace_bytes", "bsa_mask_to_lists", "bsa_prefill_mask",
-           "bsa_validate_lists"]
+           "bsa_validate_lists", "bsa_score_group_workspace_bytes", "stem_score_group", "bsa_prefill_group"]
 
 
 class BsaError(RuntimeError):
@@ -54,9 +54,13 @@ def lib():
     L.bsa_score_workspace_bytes.argtypes = [i32, i32, i32, i32, i32]
     L.bsa_score_workspace_bytes.restype = ctypes.c_size_t
     L.stem_score.argtypes = [T, T, T, i32, i32, i32, i32, i32, i32, i32, f32, P, i32, P, ctypes.c_size_t, P]
+    L.stem_score_group.argtypes = L.stem_score.argtypes
+    L.bsa_score_group_workspace_bytes.argtypes = [i32, i32, i32, i32, i32]
+    L.bsa_score_group_workspace_bytes.restype = ctypes.c_size_t
     L.stem_score_noalloc.argtypes = [T, T, T, i32, i32, i32, i32, i32, i32, i32, f32, P, i32, P]
     L.stem_select.argtypes = [P, i32, i32, P, i32, f64, f64, P, P, i64, P]
     L.bsa_prefill.argtypes = [T, T, T, T, i32, i32, i32, i32, i32, i32, P, i32, P, i64, f32, P, P]
+    L.bsa_prefill_group.argtypes = L.bsa_prefill.argtypes
     L.bsa_prefill_paged.argtypes = [T, T, P, P, i32, T, T, i32, i32, P, i32, i32, i32, i32, i32, P, i32, P, i64,
                                     f32, P, P]
     L.bsa_mask_workspace_bytes.argtypes = [i32, i32, i32]
@@ -67,7 +71,7 @@ def lib():
     L.bsa_last_error.restype = ctypes.c_char_p
     L.bsa_check_device_error.argtypes = [P]
     L.bsa_selftest_wait_timeout.argtypes = [ctypes.c_uint64, P]
-    for name in ["stem_score", "stem_score_noalloc", "stem_select", "bsa_prefill", "bsa_prefill_paged", "bsa_check_device_error",
+    for name in ["stem_score", "stem_score_group", "bsa_prefill_group", "stem_score_noalloc", "stem_select", "bsa_prefill", "bsa_prefill_paged", "bsa_check_device_error",
                  "bsa_selftest_wait_timeout", "bsa_mask_to_lists", "bsa_prefill_mask", "bsa_validate_lists"]:
         getattr(L, name).restype = ctypes.c_int
     _lib = L
@@ -146,6 +150,30 @@ def stem_score(q, k, v, block: int, metric: int = BSA_METRIC_OAM, softmax_scale:
     return scores
 
 
+def bsa_score_group_workspace_bytes(B, Hq, Hkv, nb, d) -> int:
+    return int(lib().bsa_score_group_workspace_bytes(B, Hq, Hkv, nb, d))
+
+
+def stem_score_group(q, k, v, block: int, metric: int = BSA_METRIC_OAM, softmax_scale: float = 0.0, scores=None,
+                     nb_stride: int | None = None, workspace=None, q_scale=1.0, k_scale=1.0, v_scale=1.0):
+    """Group-shared block scores [B, Hkv, nb_stride, nb_stride] fp32: one row per KV-head group,
+    from the mean of the group's query heads' pooled Q (causal lower triangle valid)."""
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    nb = (N + block - 1) // block
+    nbs = nb if nb_stride is None else nb_stride
+    if scores is None:
+        scores = torch.empty(B, Hkv, nbs, nbs, dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(bsa_score_group_workspace_bytes(B, Hq, Hkv, nb, d), dtype=torch.uint8,
+                                device=q.device)
+    st = lib().stem_score_group(tensor_arg(q, q_scale), tensor_arg(k, k_scale), tensor_arg(v, v_scale), B, N, Hq,
+                                Hkv, d, block, metric, float(softmax_scale), _ptr(scores), nbs, _ptr(workspace),
+                                workspace.numel(), _stream(q))
+    _check(st)
+    return scores
+
+
 def stem_score_noalloc(q, k, v, block: int, metric: int = BSA_METRIC_OAM, softmax_scale: float = 0.0,
                        scores=None, nb_stride: int | None = None, q_scale=1.0, k_scale=1.0, v_scale=1.0):
     """stem_score with the library's fixed 32 MiB scratch instead of a workspace (for callers
@@ -191,6 +219,25 @@ def bsa_prefill(q, k, v, block: int, row_ptr, col_idx, softmax_scale: float = 0.
     st = lib().bsa_prefill(tensor_arg(q, q_scale), tensor_arg(k, k_scale), tensor_arg(v, v_scale), tensor_arg(out),
                            B, N, Hq, Hkv, d, block, _ptr(row_ptr), row_ptr.shape[-1], _ptr(col_idx),
                            col_idx.shape[-1], float(softmax_scale), _ptr(lse), _stream(q))
+    _check(st)
+    return (out, lse) if return_lse else out
+
+
+def bsa_prefill_group(q, k, v, block: int, row_ptr, col_idx, softmax_scale: float = 0.0, out=None, lse=None,
+                      return_lse: bool = False, q_scale=1.0, k_scale=1.0, v_scale=1.0):
+    """Block-sparse causal prefill with one list per KV-head group: col_idx [B, Hkv, max_k] (from
+    stem_select on stem_score_group's scores), shared by the group's query heads."""
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    if col_idx.shape[1] != Hkv:
+        raise ValueError("col_idx must be [B, Hkv, max_k]: one list per KV-head group")
+    if out is None:
+        out = torch.empty(B, N, Hq, d, dtype=torch.bfloat16, device=q.device)
+    if return_lse and lse is None:
+        lse = torch.empty(B, Hq, N, dtype=torch.float32, device=q.device)
+    st = lib().bsa_prefill_group(tensor_arg(q, q_scale), tensor_arg(k, k_scale), tensor_arg(v, v_scale),
+                                 tensor_arg(out), B, N, Hq, Hkv, d, block, _ptr(row_ptr), row_ptr.shape[-1],
+                                 _ptr(col_idx), col_idx.shape[-1], float(softmax_scale), _ptr(lse), _stream(q))
     _check(st)
     return (out, lse) if return_lse else out
 

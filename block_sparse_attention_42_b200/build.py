@@ -12,7 +12,7 @@ ROOT = PKG.parent
 CSRC = PKG / "csrc"
 LIB = PKG / "libbsa.so"
 BUILD = ROOT / "_build"
-SOURCES = ["abi.cu", "pool.cu", "score.cu", "score_tc.cu", "select.cu", "attn.cu", "attn_ws2.cu", "attn_ws3.cu", "noalloc.cu", "selftest.cu", "mask.cu", "validate.cu"]
+SOURCES = ["abi.cu", "pool.cu", "score.cu", "score_tc.cu", "select.cu", "attn.cu", "attn_ws2.cu", "attn_ws3.cu", "attn_group.cu", "noalloc.cu", "selftest.cu", "mask.cu", "validate.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-std=c++17", "-lineinfo",
          "-Xcompiler", "-fPIC", "-Xptxas", "-v", f"-I{ROOT / 'include'}", f"-I{CSRC}"]

@@ -206,7 +206,7 @@ bsa_status_t prefill_launch(const bsa_tensor_t& q, const bsa_tensor_t& k, const 
                             const bsa_tensor_t& out, int32_t B, int32_t N, int32_t Hq, int32_t Hkv, int32_t d,
                             int32_t block, const int32_t* row_ptr, int32_t row_ptr_stride, int32_t row_ptr_hstride,
                             int32_t allow_empty, const int32_t* col_idx, int64_t max_k, float softmax_scale,
-                            float* lse, cudaStream_t stream) {
+                            float* lse, cudaStream_t stream, bool group = false) {
     bsa_status_t st;
     const int nb = (N + block - 1) / block;
     bsa_status_t est;
@@ -246,7 +246,14 @@ bsa_status_t prefill_launch(const bsa_tensor_t& q, const bsa_tensor_t& k, const 
     a.lse = lse;
     a.lse_stride = N;
     a.err = err;
-    cudaError_t e = launch_attn(fp8, false, tq, tk, tv, a, stream);
+    a.list_per_group = group ? 1 : 0;
+    // Group-shared lists: the GQA-packed kernel where it applies (BSA_ATTN_VARIANT still picks a
+    // per-head kernel for cross-checks), else the per-head kernels on the shared lists.
+    const char* var = std::getenv("BSA_ATTN_VARIANT");
+    const bool packed = group && attention_group_packed(fp8, a) && (!var || std::strcmp(var, "group") == 0);
+    cudaError_t e = packed
+                        ? launch_attention_group(fp8, false, tq, tk, tv, a, stream)
+                        : launch_attn(fp8, false, tq, tk, tv, a, stream);
     if (e != cudaSuccess) return cuda_fail(e, "bsa_prefill launch");
     return BSA_OK;
 }
@@ -342,10 +349,23 @@ size_t bsa_score_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int32_t nb,
            2 * align256(sizeof(float) * size_t(B) * Hkv * nb * d) + align256(sizeof(float) * size_t(B) * Hkv * nb);
 }
 
-bsa_status_t stem_score(bsa_tensor_t q, bsa_tensor_t k, bsa_tensor_t v, int32_t B, int32_t N, int32_t Hq,
-                        int32_t Hkv, int32_t d, int32_t block, int32_t metric, float softmax_scale, float* scores,
-                        int32_t nb_stride, void* ws, size_t ws_bytes, cudaStream_t stream) {
-    NvtxRange nvtx_range("stem_score");
+size_t bsa_score_group_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int32_t nb, int32_t d) {
+    const size_t base = bsa_score_workspace_bytes(B, Hq, Hkv, nb, d);
+    if (base == 0) return 0;
+    return base + 2 * align256(sizeof(float) * size_t(B) * Hkv * nb * d);
+}
+
+}  // extern "C"
+
+namespace bsa {
+namespace {
+
+// stem_score and stem_score_group: pool (a1), then the score GEMM (a2) with one query row per
+// query head, or (group) one per KV-head group from the group mean of the heads' pooled Q.
+bsa_status_t score_common(bool group, const bsa_tensor_t& q, const bsa_tensor_t& k, const bsa_tensor_t& v, int32_t B,
+                          int32_t N, int32_t Hq, int32_t Hkv, int32_t d, int32_t block, int32_t metric,
+                          float softmax_scale, float* scores, int32_t nb_stride, void* ws, size_t ws_bytes,
+                          cudaStream_t stream) {
     bsa_status_t st;
     if ((st = check_tensor(q, "q", B > 1)) || (st = check_tensor(k, "k", B > 1)) || (st = check_tensor(v, "v", B > 1)))
         return st;
@@ -359,12 +379,14 @@ bsa_status_t stem_score(bsa_tensor_t q, bsa_tensor_t k, bsa_tensor_t v, int32_t 
     if (B > 65535 || Hq > 65535) return fail(BSA_ERR_UNSUPPORTED, "B and Hq must be <= 65535");
     if (!scores) return fail(BSA_ERR_INVALID_ARG, "scores is null");
     if (nb_stride < nb) return fail(BSA_ERR_INVALID_ARG, "nb_stride (%d) < number of blocks (%d)", nb_stride, nb);
-    const size_t need = bsa_score_workspace_bytes(B, Hq, Hkv, nb, d);
+    const size_t need = group ? bsa_score_group_workspace_bytes(B, Hq, Hkv, nb, d)
+                              : bsa_score_workspace_bytes(B, Hq, Hkv, nb, d);
     if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u))
         return fail(BSA_ERR_WORKSPACE, "workspace must be >= %zu bytes and 256-byte aligned", need);
-    // Workspace: [qhi | qlo | khi | klo | vbar], each part 256-byte aligned.
+    // Workspace: [qhi | qlo | khi | klo | vbar (| ghi | glo)], each part 256-byte aligned.
     const size_t qbytes = align256(sizeof(float) * size_t(B) * Hq * nb * d);
     const size_t kbytes = align256(sizeof(float) * size_t(B) * Hkv * nb * d);
+    const size_t vbytes = align256(sizeof(float) * size_t(B) * Hkv * nb);
     char* w = static_cast<char*>(ws);
     float* qhi = reinterpret_cast<float*>(w);
     float* qlo = reinterpret_cast<float*>(w + qbytes);
@@ -376,27 +398,58 @@ bsa_status_t stem_score(bsa_tensor_t q, bsa_tensor_t k, bsa_tensor_t v, int32_t 
     cudaError_t e =
         launch_pool(dt, targ(q), targ(k), targ(v), B, N, Hq, Hkv, d, block, qhi, qlo, khi, klo, vbar, stream);
     if (e != cudaSuccess) return cuda_fail(e, "pool launch");
+    int Hrows = Hq;  // query-side heads of the score GEMM
+    if (group) {
+        float* ghi = reinterpret_cast<float*>(w + 2 * qbytes + 2 * kbytes + vbytes);
+        float* glo = reinterpret_cast<float*>(w + 2 * qbytes + 3 * kbytes + vbytes);
+        e = launch_group_mean(qhi, qlo, B, Hq, Hkv, nb, d, ghi, glo, stream);
+        if (e != cudaSuccess) return cuda_fail(e, "group mean launch");
+        qhi = ghi;
+        qlo = glo;
+        Hrows = Hkv;
+    }
     // Score GEMM on the tensor cores (3xTF32, score_tc.cu); BSA_SCORE_VARIANT=simt selects the
     // fp32 FMA kernel (score.cu), which computes the same scores to fp32 rounding.
     const char* sv = std::getenv("BSA_SCORE_VARIANT");
     if (sv && std::strcmp(sv, "simt") == 0) {
-        e = launch_score(qhi, qlo, khi, klo, vbar, B, Hq, Hkv, nb, d, tau, metric, scores, nb_stride, stream);
+        e = launch_score(qhi, qlo, khi, klo, vbar, B, Hrows, Hkv, nb, d, tau, metric, scores, nb_stride, stream);
     } else {
         bsa_status_t est;
         unsigned* err = device_error_word(&est);
         if (err == nullptr) return est;
         CUtensorMap mqh, mql, mkh, mkl;
         const int64_t ro = d, qh = int64_t(nb) * d, kh = int64_t(nb) * d;
-        if ((st = make_map(&mqh, qhi, 4, d, nb, Hq, B, ro, qh, qh * Hq, 128, "qhi")) ||
-            (st = make_map(&mql, qlo, 4, d, nb, Hq, B, ro, qh, qh * Hq, 128, "qlo")) ||
+        if ((st = make_map(&mqh, qhi, 4, d, nb, Hrows, B, ro, qh, qh * Hrows, 128, "qhi")) ||
+            (st = make_map(&mql, qlo, 4, d, nb, Hrows, B, ro, qh, qh * Hrows, 128, "qlo")) ||
             (st = make_map(&mkh, khi, 4, d, nb, Hkv, B, ro, kh, kh * Hkv, 128, "khi")) ||
             (st = make_map(&mkl, klo, 4, d, nb, Hkv, B, ro, kh, kh * Hkv, 128, "klo")))
             return st;
-        e = launch_score_tc(mqh, mql, mkh, mkl, vbar, B, Hq, Hkv, nb, d, tau, metric, scores, nb_stride, err,
+        e = launch_score_tc(mqh, mql, mkh, mkl, vbar, B, Hrows, Hkv, nb, d, tau, metric, scores, nb_stride, err,
                             stream);
     }
     if (e != cudaSuccess) return cuda_fail(e, "score launch");
     return BSA_OK;
+}
+
+}  // namespace
+}  // namespace bsa
+
+extern "C" {
+
+bsa_status_t stem_score(bsa_tensor_t q, bsa_tensor_t k, bsa_tensor_t v, int32_t B, int32_t N, int32_t Hq,
+                        int32_t Hkv, int32_t d, int32_t block, int32_t metric, float softmax_scale, float* scores,
+                        int32_t nb_stride, void* ws, size_t ws_bytes, cudaStream_t stream) {
+    NvtxRange nvtx_range("stem_score");
+    return score_common(false, q, k, v, B, N, Hq, Hkv, d, block, metric, softmax_scale, scores, nb_stride, ws,
+                        ws_bytes, stream);
+}
+
+bsa_status_t stem_score_group(bsa_tensor_t q, bsa_tensor_t k, bsa_tensor_t v, int32_t B, int32_t N, int32_t Hq,
+                              int32_t Hkv, int32_t d, int32_t block, int32_t metric, float softmax_scale,
+                              float* scores, int32_t nb_stride, void* ws, size_t ws_bytes, cudaStream_t stream) {
+    NvtxRange nvtx_range("stem_score_group");
+    return score_common(true, q, k, v, B, N, Hq, Hkv, d, block, metric, softmax_scale, scores, nb_stride, ws,
+                        ws_bytes, stream);
 }
 
 bsa_status_t stem_select(const float* scores, int32_t B, int32_t Hq, const int32_t* nb_per_seq, int32_t nb_stride,
@@ -437,6 +490,19 @@ bsa_status_t bsa_prefill(bsa_tensor_t q, bsa_tensor_t k, bsa_tensor_t v, bsa_ten
     if (row_ptr_stride < nb + 1) return fail(BSA_ERR_INVALID_ARG, "row_ptr_stride must be >= nb + 1");
     return prefill_launch(q, k, v, out, B, N, Hq, Hkv, d, block, row_ptr, row_ptr_stride, 0, 0, col_idx, max_k,
                           softmax_scale, lse, stream);
+}
+
+bsa_status_t bsa_prefill_group(bsa_tensor_t q, bsa_tensor_t k, bsa_tensor_t v, bsa_tensor_t out, int32_t B,
+                               int32_t N, int32_t Hq, int32_t Hkv, int32_t d, int32_t block, const int32_t* row_ptr,
+                               int32_t row_ptr_stride, const int32_t* col_idx, int64_t max_k, float softmax_scale,
+                               float* lse, cudaStream_t stream) {
+    NvtxRange nvtx_range("bsa_prefill_group");
+    bsa_status_t st;
+    if ((st = prefill_checks(q, k, v, out, B, N, Hq, Hkv, d, block, row_ptr, col_idx, max_k))) return st;
+    const int nb = (N + block - 1) / block;
+    if (row_ptr_stride < nb + 1) return fail(BSA_ERR_INVALID_ARG, "row_ptr_stride must be >= nb + 1");
+    return prefill_launch(q, k, v, out, B, N, Hq, Hkv, d, block, row_ptr, row_ptr_stride, 0, 0, col_idx, max_k,
+                          softmax_scale, lse, stream, true);
 }
 
 size_t bsa_mask_workspace_bytes(int32_t B, int32_t Hq, int32_t nb) {

@@ -118,7 +118,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int32_t* rp = a.row_ptr + static_cast<int64_t>(b) * a.row_ptr_stride + static_cast<int64_t>(h) * a.row_ptr_hstride;
     const int l_begin = rp[i];
     const int n_list = rp[i + 1] - l_begin;
-    const int32_t* gl = a.col_idx + (static_cast<int64_t>(b) * a.Hq + h) * a.max_k + l_begin;
+    const int64_t lrow = a.list_per_group ? static_cast<int64_t>(b) * a.Hkv + h / (a.Hq / a.Hkv)
+                                          : static_cast<int64_t>(b) * a.Hq + h;
+    const int32_t* gl = a.col_idx + lrow * a.max_k + l_begin;
     bool bad = n_list < 1 || n_list > kMaxBlocks || l_begin < 0 || l_begin + static_cast<int64_t>(n_list) > a.max_k;
     const int n_use = bad ? 0 : n_list;
     for (int n = tid; n < n_use; n += kThreads) {

@@ -56,9 +56,13 @@ __device__ __forceinline__ int physical_page(const AttnArgs& a, int b, int lp, i
     return phys;
 }
 
-// List entry n of the tile; -1 if out of [0, i] (skipped block: scores all -inf).
+// List entry n of the tile; -1 if out of [0, i] (skipped block: scores all -inf).  The lists
+// are per query head (col_idx [B, Hq, max_k]) or, for group-shared selection, per KV head
+// (col_idx [B, Hkv, max_k]).
 __device__ __forceinline__ int list_entry(const AttnArgs& a, const Tile& T, int n) {
-    const int j = __ldg(a.col_idx + (static_cast<int64_t>(T.b) * a.Hq + T.h) * a.max_k + T.l_begin + n);
+    const int64_t row = a.list_per_group ? static_cast<int64_t>(T.b) * a.Hkv + T.hk
+                                         : static_cast<int64_t>(T.b) * a.Hq + T.h;
+    const int j = __ldg(a.col_idx + row * a.max_k + T.l_begin + n);
     return (j >= 0 && j <= T.i) ? j : -1;
 }
 

@@ -28,6 +28,11 @@ struct TensorArg {
 cudaError_t launch_pool(int dtype, TensorArg q, TensorArg k, TensorArg v, int B, int N, int Hq, int Hkv, int d,
                         int block, float* qhi, float* qlo, float* khi, float* klo, float* vbar, cudaStream_t s);
 
+// a1, group-shared selection: ghi + glo [B, Hkv, nb, d] = mean over the G = Hq / Hkv query heads
+// of each KV-head group of qhi + qlo [B, Hq, nb, d] (fp64 sum, one fp32 rounding, hi / lo split).
+cudaError_t launch_group_mean(const float* qhi, const float* qlo, int B, int Hq, int Hkv, int nb, int d, float* ghi,
+                              float* glo, cudaStream_t s);
+
 // a2: block scores from pooled representations.
 // tcgen05 3xTF32 GEMM (score_tc.cu) over 4-D tensor maps of qhi, qlo [d, nb, Hq, B] and khi,
 // klo [d, nb, Hkv, B] (fp32, 128-byte swizzle, box 32 x 128); err = device error word.
@@ -61,8 +66,9 @@ struct AttnArgs {
     int row_ptr_hstride;         // entries between query heads (0: one row_ptr for all heads)
     int allow_empty;             // 1: an empty list is a row with no kept block (its output
                                  // is written elsewhere), not an error
-    const int32_t* col_idx;
+    const int32_t* col_idx;      // [B, Hq, max_k], or [B, Hkv, max_k] with list_per_group
     int64_t max_k;
+    int list_per_group;          // 1: one list per KV-head group, shared by its query heads
     const int32_t* page_table;   // paged only
     int max_pages, page_size, num_pages;
     float scale_log2;            // softmax scale * log2(e) (* q_scale * k_scale for FP8)
@@ -82,6 +88,12 @@ cudaError_t launch_attention_ws2(bool fp8, bool paged, const CUtensorMap& tq, co
 // on block k (attn_ws3.cu).  FP8, and BF16 shapes whose stages fit two CTAs per SM.
 cudaError_t launch_attention_ws3(bool fp8, bool paged, const CUtensorMap& tq, const CUtensorMap& tk,
                                  const CUtensorMap& tv, const AttnArgs& a, cudaStream_t s);
+// Group-shared lists (a.list_per_group): one CTA per SM serves two query heads of a KV-head group
+// for a query block, loading each kept K/V block once for both (attn_group.cu).  Applies to FP8
+// at d = 128 / block 128 with an even group size (attention_group_packed).
+bool attention_group_packed(bool fp8, const AttnArgs& a);
+cudaError_t launch_attention_group(bool fp8, bool paged, const CUtensorMap& tq, const CUtensorMap& tk,
+                                   const CUtensorMap& tv, const AttnArgs& a, cudaStream_t s);
 
 // Block mask -> per-head CSR lists (mask.cu).  mask [B, Hq, nb, mask_stride] uint8 (16-byte
 // aligned, mask_stride a multiple of 16 and >= nb); row_ptr [B*Hq][nb+1]; col_idx [B*Hq][cap]

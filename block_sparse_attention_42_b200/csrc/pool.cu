@@ -262,7 +262,40 @@ __global__ void __launch_bounds__(kPoolThreads, DT == 1 ? 4 : 2) pool_kernel(con
     }
 }
 
+// Group-shared selection: the mean over the G query heads of a KV-head group of their pooled
+// Q means, as hi + lo like the per-head means.  One thread per output element; each head's mean
+// is read as hi + lo (exactly the fp32 mean) and the G of them are summed in fp64, so the group
+// mean carries one final fp32 rounding.
+__global__ void __launch_bounds__(256) group_mean_kernel(const float* __restrict__ qhi, const float* __restrict__ qlo,
+                                                         int B, int Hq, int Hkv, int nb, int d,
+                                                         float* __restrict__ ghi, float* __restrict__ glo) {
+    const int64_t n_out = static_cast<int64_t>(B) * Hkv * nb * d;
+    const int64_t o = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (o >= n_out) return;
+    const int G = Hq / Hkv;
+    const int64_t per_head = static_cast<int64_t>(nb) * d;
+    const int64_t bk = o / per_head, rest = o % per_head;  // bk = b * Hkv + hk
+    const int64_t b = bk / Hkv, hk = bk % Hkv;
+    double acc = 0.0;
+    for (int g = 0; g < G; ++g) {
+        const int64_t src = (b * Hq + hk * G + g) * per_head + rest;
+        acc += static_cast<double>(qhi[src]) + static_cast<double>(qlo[src]);
+    }
+    const float m = static_cast<float>(acc / G);
+    const float hi = __uint_as_float(__float_as_uint(m) & 0xFFFFE000u);
+    ghi[o] = hi;
+    glo[o] = isfinite(m) ? m - hi : 0.f;
+}
+
 }  // namespace
+
+cudaError_t launch_group_mean(const float* qhi, const float* qlo, int B, int Hq, int Hkv, int nb, int d, float* ghi,
+                              float* glo, cudaStream_t s) {
+    const int64_t n = static_cast<int64_t>(B) * Hkv * nb * d;
+    const unsigned blocks = static_cast<unsigned>((n + 255) / 256);
+    group_mean_kernel<<<blocks, 256, 0, s>>>(qhi, qlo, B, Hq, Hkv, nb, d, ghi, glo);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_pool(int dtype, TensorArg q, TensorArg k, TensorArg v, int B, int N, int Hq, int Hkv, int d,
                         int block, float* qbar, float* qlo, float* kbar, float* klo, float* vbar, cudaStream_t s) {

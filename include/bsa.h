@@ -124,6 +124,38 @@ bsa_status_t bsa_prefill(bsa_tensor_t q, bsa_tensor_t k, bsa_tensor_t v, bsa_ten
                          const int32_t* row_ptr, int32_t row_ptr_stride, const int32_t* col_idx,
                          int64_t max_k, float softmax_scale, float* lse, cudaStream_t stream);
 
+/* Group-shared selection with GQA-packed attention.  The pages select per query head and say
+ * nothing about grouped-query attention.  This extension gives the G = Hq / Hkv query heads of
+ * a KV-head group one kept-block list, so that the heads sharing a list can share every K/V
+ * load [a reading of cn486 page, §二.2.2 BSA算子优化: the list is built before the inner loop,
+ * which then only visits valid blocks].
+ *
+ * stem_score_group: stem_score with one score row per KV-head group.  The query-side
+ * representation is the mean over the group's G heads of their pooled Q:
+ *     scores[b, hk, i, j] = tau * Gbar[b,hk,i] . Kbar[b,hk,j]  (+ ln vbar[b,hk,j] for OAM),
+ *     Gbar[b,hk,i] = (1/G) * sum over the heads h of group hk of Qbar[b,h,i],
+ * which is the mean of the G heads' stem_score rows (every metric is linear in Qbar).
+ * scores is fp32 [B, Hkv, nb_stride, nb_stride]; ws needs bsa_score_group_workspace_bytes()
+ * bytes, 256-byte aligned.  Arguments and errors otherwise as in stem_score.  stem_select then
+ * runs on these scores with Hq := Hkv and writes col_idx [B, Hkv, max_k].
+ *
+ * bsa_prefill_group: bsa_prefill whose col_idx is [B, Hkv, max_k], one list per KV-head group,
+ * shared by the group's query heads (row_ptr as stem_select writes it).  FP8 at d = 128, block
+ * 128, with G even, runs the GQA-packed kernel: one CTA serves two query heads of a group for a
+ * query block and loads each kept K/V block once for both.  Every other shape runs the per-head
+ * kernel on the shared lists.  Arguments, outputs and errors otherwise as in bsa_prefill.
+ * bsa_score_group_workspace_bytes returns 0 for invalid sizes. */
+size_t bsa_score_group_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int32_t nb, int32_t d);
+bsa_status_t stem_score_group(bsa_tensor_t q, bsa_tensor_t k, bsa_tensor_t v, int32_t B, int32_t N,
+                              int32_t Hq, int32_t Hkv, int32_t d, int32_t block, int32_t metric,
+                              float softmax_scale, float* scores, int32_t nb_stride, void* ws,
+                              size_t ws_bytes, cudaStream_t stream);
+bsa_status_t bsa_prefill_group(bsa_tensor_t q, bsa_tensor_t k, bsa_tensor_t v, bsa_tensor_t out,
+                               int32_t B, int32_t N, int32_t Hq, int32_t Hkv, int32_t d,
+                               int32_t block, const int32_t* row_ptr, int32_t row_ptr_stride,
+                               const int32_t* col_idx, int64_t max_k, float softmax_scale,
+                               float* lse, cudaStream_t stream);
+
 /* Block-mask input [cn486 page, §二.2.2 BSA算子优化: the sparse kernel receives the selection
  * as a block mask and derives the kept-block list from it before its inner loop].
  * block_mask (device, uint8) is [B, Hq, nb, mask_stride] with nb = ceil(N / block): row
