@@ -76,6 +76,8 @@ def _load():
                                        ctypes.c_int, P, i64, ctypes.c_int]
     lib.orc_effective_flop.restype = f64
     lib.orc_set_threads.argtypes = [ctypes.c_int]
+    lib.orc_attention_rows_skip.argtypes = [T, T, T, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                            ctypes.c_int, P, ctypes.c_int, P, i64, f64, f64, P, i64, P, P, P]
     lib.orc_group_mean.argtypes = [P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, P]
     _lib = lib
     return lib
@@ -219,6 +221,24 @@ def attention_rows(q: View, k: View, v: View, N, Hq, Hkv, D, bs, row_ptr, col_id
                                col_idx.shape[-1], float(tau), _ptr(rows), n, _ptr(out), _ptr(lse),
                                None if amp is None else _ptr(amp))
     return (out, lse, amp) if with_amp else (out, lse)
+
+
+def attention_rows_skip(q: View, k: View, v: View, N, Hq, Hkv, D, bs, row_ptr, col_idx, tau, lam: float, rows):
+    """O, LSE and the number of skipped list blocks of the requested (b, h, t) rows under the
+    threshold skip with parameter lam (0 skips nothing), fp64."""
+    row_ptr = _c(row_ptr, np.int32)
+    col_idx = _c(col_idx, np.int32)
+    rows = _c(rows, np.int64).reshape(-1, 3)
+    n = rows.shape[0]
+    out = np.empty((n, D), np.float64)
+    lse = np.empty((n,), np.float64)
+    skipped = np.empty((n,), np.int32)
+    ln_lam = float(np.log(lam)) if lam > 0 else -np.inf
+    _load().orc_attention_rows_skip(ctypes.byref(q.struct), ctypes.byref(k.struct), ctypes.byref(v.struct),
+                                    N, Hq, Hkv, D, bs, _ptr(row_ptr), row_ptr.shape[-1], _ptr(col_idx),
+                                    col_idx.shape[-1], float(tau), ln_lam, _ptr(rows), n, _ptr(out), _ptr(lse),
+                                    _ptr(skipped))
+    return out, lse, skipped
 
 
 def attention_rows_mask(q: View, k: View, v: View, N, Hq, Hkv, D, bs, mask, tau, rows,

@@ -10,6 +10,8 @@
  *        §3.1 Token位置衰减策略（TPD）, §3.2 输出感知度量（OAM）,
  *        §二.2.1 Stem算子优化 (pooled block representations + one GEMM; fused budget+sort),
  *        §二.2.2 BSA算子优化 (skipped block == all scores -inf).
+ *   [P5] "BLASST: Dynamic BLocked Attention Sparsity via Softmax Thresholding" (gist.science):
+ *        §2.1 (skip a block whose local max trails the running max by more than ln(lambda)).
  *   [P4] "Tencent Hunyuan introduces Stem sparse attention algorithm" (setupai.cc):
  *        "Technical Deep Dive" (TPD: position-dependent top-k, more budget to early
  *        positions; OAM: approximate output magnitude using value information).
@@ -36,6 +38,9 @@
  *   orc_attention_rows  pinned: density 1 == library dense causal SDPA (fp64); skipped
  *                       blocks' contents are irrelevant; single-key closed form.  Its amp
  *                       output == library SDPA with |V| as the values; single key: |v|.
+ *   orc_attention_rows_skip  pinned: lambda = 0 gives orc_attention_rows exactly; a block whose
+ *                       max trails by more / less than ln(lambda) is skipped / kept (closed
+ *                       form); with its skip decisions, == library SDPA under the per-row mask.
  *   orc_attention_rows_mask  pinned: an all-ones mask == library dense causal SDPA; a
  *                       diagonal-only mask == library SDPA over the block's own keys; an
  *                       empty row gives 0 / -inf; entries above the diagonal are ignored.
@@ -438,6 +443,72 @@ void orc_attention_rows(const orc_tensor* q, const orc_tensor* k, const orc_tens
             if (a)
                 for (int c = 0; c < D; ++c) a[c] /= z;
             if (lse) lse[r] = m + log(z);
+        }
+        free(allowed);
+        free(logit);
+        free(qrow);
+    }
+}
+
+/* Attention with the threshold skip of [P5] ("BLASST: Dynamic BLocked Attention Sparsity via
+ * Softmax Thresholding", §2.1 基于运行最大值的剪枝) on top of the kept-block lists.  For query
+ * token t the list's blocks are visited in stored order while a running maximum m of the logits
+ * seen so far is kept: for block j, with m~ the largest logit tau * q_t . k_s over its allowed
+ * keys s <= t, the block is skipped when m is finite and m~ - m < ln(lambda); otherwise its keys
+ * join the softmax and m = max(m, m~).  A skipped block contributes nothing.  O and lse are
+ * those of the softmax over the keys of the blocks that were not skipped.  skipped (nullable)
+ * receives, per row, the number of list blocks skipped.  ln_lambda = -inf skips nothing. */
+void orc_attention_rows_skip(const orc_tensor* q, const orc_tensor* k, const orc_tensor* v, int N,
+                             int Hq, int Hkv, int D, int bs, const int32_t* row_ptr, int rp_stride,
+                             const int32_t* col_idx, int64_t maxK, double tau, double ln_lambda,
+                             const int64_t* rows, int64_t n_rows, double* out /* [n_rows][D] */,
+                             double* lse /* [n_rows] */, int32_t* skipped /* nullable [n_rows] */) {
+    int G = Hq / Hkv;
+#pragma omp parallel
+    {
+        unsigned char* allowed = (unsigned char*)malloc((size_t)N);
+        double* logit = (double*)malloc(sizeof(double) * (size_t)N);
+        double* qrow = (double*)malloc(sizeof(double) * (size_t)D);
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t r = 0; r < n_rows; ++r) {
+            int64_t b = rows[3 * r], h = rows[3 * r + 1], t = rows[3 * r + 2];
+            int64_t hk = h / G;
+            int64_t i = t / bs;
+            const int32_t* rp = &row_ptr[b * rp_stride];
+            const int32_t* list = &col_idx[(b * Hq + h) * maxK + rp[i]];
+            int32_t len = rp[i + 1] - rp[i];
+            for (int c = 0; c < D; ++c) qrow[c] = load_elem(q, b, t, h, c);
+            memset(allowed, 0, (size_t)N);
+            double m = -INFINITY;
+            int32_t n_skip = 0;
+            for (int32_t n = 0; n < len; ++n) {
+                int64_t j = list[n];
+                double mb = -INFINITY;
+                for (int64_t s = j * bs; s < (j + 1) * bs && s < N && s <= t; ++s) {
+                    double dot = 0.0;
+                    for (int c = 0; c < D; ++c) dot += qrow[c] * load_elem(k, b, s, hk, c);
+                    logit[s] = tau * dot;
+                    if (logit[s] > mb) mb = logit[s];
+                }
+                if (m > -INFINITY && mb - m < ln_lambda) {
+                    ++n_skip;
+                    continue;
+                }
+                for (int64_t s = j * bs; s < (j + 1) * bs && s < N && s <= t; ++s) allowed[s] = 1;
+                if (mb > m) m = mb;
+            }
+            double z = 0.0;
+            double* o = &out[r * D];
+            for (int c = 0; c < D; ++c) o[c] = 0.0;
+            for (int64_t s = 0; s <= t; ++s) {
+                if (!allowed[s]) continue;
+                double w = exp(logit[s] - m);
+                z += w;
+                for (int c = 0; c < D; ++c) o[c] += w * load_elem(v, b, s, hk, c);
+            }
+            for (int c = 0; c < D; ++c) o[c] /= z;
+            if (lse) lse[r] = m + log(z);
+            if (skipped) skipped[r] = n_skip;
         }
         free(allowed);
         free(logit);

@@ -390,6 +390,60 @@ def test_single_key_closed_form(orc):
     assert np.array_equal(amp[0], np.abs(v[0, 0, 0]))
 
 
+# ----------------------------------------------------------------------------- threshold skip
+
+
+def test_skip_with_lambda_zero_is_plain_attention(orc):
+    w = inputs.Workload("pin", 1, 4, 2, 96, 16, 8, "fp32", 0.4, "stem", 94)
+    d = inputs.make_inputs(w)
+    q, k, v = d["q"].double(), d["k"].double(), d["v"].double()
+    B, N, Hq, Hkv, D, bs = 1, 96, 4, 2, 16, 8
+    nb = N // bs
+    S = np.random.default_rng(8).standard_normal((B, Hq, nb, nb))
+    rp, ci = orc.select(S, [nb], 0.4)
+    rows = _all_rows(B, Hq, N)
+    ref, ref_lse = orc.attention_rows(orc.view(q), orc.view(k), orc.view(v), N, Hq, Hkv, D, bs, rp, ci, 0.3, rows)
+    out, lse, skipped = orc.attention_rows_skip(orc.view(q), orc.view(k), orc.view(v), N, Hq, Hkv, D, bs, rp, ci,
+                                                0.3, 0.0, rows)
+    assert np.array_equal(out, ref) and np.array_equal(lse, ref_lse) and not skipped.any()
+    # the number of skipped blocks never falls as lambda grows
+    prev = np.zeros_like(skipped)
+    for lam in (1e-6, 1e-3, 1e-1, 0.5, 1.0):
+        _, _, sk = orc.attention_rows_skip(orc.view(q), orc.view(k), orc.view(v), N, Hq, Hkv, D, bs, rp, ci, 0.3,
+                                           lam, rows)
+        assert np.all(sk >= prev)
+        prev = sk
+    assert prev.any()
+
+
+def test_skip_closed_form():
+    """Two blocks of 8 keys.  Block 0's keys all give the logit 10, block 1's keys the logit 0.
+    Row t in block 1 visits block 0 then block 1: block 1's max trails by 10, so it is skipped
+    for lambda = e^-9 (O = mean of block 0's values) and kept for lambda = e^-11 (O = the two
+    blocks weighted e^10 : 1 per key)."""
+    import oracle as orc
+    N, D, bs = 16, 4, 8
+    q = np.zeros((1, N, 1, D)); q[0, :, 0, 0] = 1.0
+    k = np.zeros((1, N, 1, D)); k[0, :8, 0, 0] = 10.0
+    v = np.random.default_rng(3).standard_normal((1, N, 1, D))
+    rp = np.array([[0, 1, 3]], np.int32)
+    ci = np.array([[[0, 0, 1]]], np.int32)
+    for t in (8, 11, 15):
+        rows = np.array([(0, 0, t)], np.int64)
+        o, lse, sk = orc.attention_rows_skip(orc.view(q), orc.view(k), orc.view(v), N, 1, 1, D, bs, rp, ci, 1.0,
+                                             math.exp(-9.0), rows)
+        assert sk[0] == 1
+        np.testing.assert_allclose(o[0], v[0, :8, 0].mean(axis=0), rtol=1e-13, atol=1e-14)
+        assert lse[0] == pytest.approx(10.0 + math.log(8.0), rel=1e-15)
+        o, lse, sk = orc.attention_rows_skip(orc.view(q), orc.view(k), orc.view(v), N, 1, 1, D, bs, rp, ci, 1.0,
+                                             math.exp(-11.0), rows)
+        n1 = t - 7
+        wts = np.array([math.exp(10.0)] * 8 + [1.0] * n1)
+        ref = (wts[:, None] * v[0, :t + 1, 0]).sum(axis=0) / wts.sum()
+        assert sk[0] == 0
+        np.testing.assert_allclose(o[0], ref, rtol=1e-13, atol=1e-14)
+
+
 # ----------------------------------------------------------------------------- block-mask input
 
 
