@@ -53,6 +53,7 @@ def parse():
     p.add_argument("--no-sweeps", action="store_true",
                    help="skip the density, length and paged-varlen sweeps of bsa_prefill")
     p.add_argument("--sweep-reps", type=int, default=3, help="timed calls per sweep point")
+    p.add_argument("--no-skip", action="store_true", help="skip the threshold-skip (bsa_prefill_skip) measurement")
     p.add_argument("--no-group", action="store_true",
                    help="skip the group-shared selection + GQA-packed attention measurement")
     return p.parse_args()
@@ -558,6 +559,29 @@ def run_ours(args, rank, world, device):
                         "per_head_bsa_prefill_ms": res["attn_ms"], "reps": reps}
         del g_scores, g_ws, g_rp, g_ci, g_out
 
+    # Threshold skip on top of the step's lists: speed and the kernel's own skip counters.
+    if not args.no_skip and rank == 0 and (fp8 or D == 64 or w.block == 64):
+        pts = []
+        reps = max(3, min(args.steps, 10))
+        for lam in (1e-4, 1e-3, 1e-2):
+            stats = torch.zeros(4, dtype=torch.int64, device=device)
+            s_out = torch.empty_like(out)
+            bsa.bsa_prefill_skip(q, k, v, w.block, row_ptr, col_idx, lam, out=s_out, skip_stats=stats, **scale_kw)
+            torch.cuda.synchronize(device)
+            st = stats.cpu().tolist()
+            ms = _time_calls(lambda: bsa.bsa_prefill_skip(q, k, v, w.block, row_ptr, col_idx, lam, out=s_out,
+                                                          **scale_kw), reps, stream)
+            diff = (s_out.float() - out.float())
+            pts.append({"lambda": lam, "ms": ms, "speedup_vs_bsa_prefill": res["attn_ms"] / ms,
+                        "row_block_skip_rate": st[1] / max(st[0], 1),
+                        "tile_block_product_skip_rate": st[3] / max(st[2], 1),
+                        "rel_l2_vs_no_skip": float(diff.norm() / out.float().norm())})
+            del s_out, stats
+        bsa.bsa_check_device_error(device)
+        res["skip"] = {"what": "bsa_prefill_skip: a row drops a kept block whose max trails its running max by more "
+                               "than ln(lambda); a warp whose rows all drop it skips the exponentials, a query block "
+                               "whose rows all drop it skips the P.V product", "reps": reps, "points": pts}
+
     if not args.no_sweeps and rank == 0:
         res["sweeps"] = run_sweeps(args, device, dict(name=w.name, q=q, k=k, v=v, scores=scores, block=w.block,
                                                       seqlens=[N] * B, scale_kw=scale_kw))
@@ -785,6 +809,8 @@ def main():
             line["sweeps"] = res["sweeps"]
         if "group" in res:
             line["group_shared"] = res["group"]
+        if "skip" in res:
+            line["threshold_skip"] = res["skip"]
         if "mask" in res:
             m = dict(res["mask"])
             m["mask_to_lists_roofline"] = {"bound": "hbm", "achieved": m.pop("mask_to_lists_gbs"),

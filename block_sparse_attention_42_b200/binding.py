@@ -25,7 +25,8 @@ STATUS = {0: "BSA_OK", 1: "BSA_ERR_INVALID_ARG", 2: "BSA_ERR_UNSUPPORTED", 3: "B
 EXPORTS = ["bsa_tpd_budget", "bsa_score_workspace_bytes", "stem_score", "stem_select", "bsa_prefill",
            "bsa_prefill_paged", "bsa_last_error", "bsa_check_device_error", "stem_score_noalloc",
            "bsa_selftest_wait_timeout", "bsa_mask_workspace_bytes", "bsa_mask_to_lists", "bsa_prefill_mask",
-           "bsa_validate_lists", "bsa_score_group_workspace_bytes", "stem_score_group", "bsa_prefill_group"]
+           "bsa_validate_lists", "bsa_score_group_workspace_bytes", "stem_score_group", "bsa_prefill_group",
+           "bsa_prefill_skip"]
 
 
 class BsaError(RuntimeError):
@@ -61,6 +62,7 @@ def lib():
     L.stem_select.argtypes = [P, i32, i32, P, i32, f64, f64, P, P, i64, P]
     L.bsa_prefill.argtypes = [T, T, T, T, i32, i32, i32, i32, i32, i32, P, i32, P, i64, f32, P, P]
     L.bsa_prefill_group.argtypes = L.bsa_prefill.argtypes
+    L.bsa_prefill_skip.argtypes = [T, T, T, T, i32, i32, i32, i32, i32, i32, P, i32, P, i64, f32, f64, P, P, P]
     L.bsa_prefill_paged.argtypes = [T, T, P, P, i32, T, T, i32, i32, P, i32, i32, i32, i32, i32, P, i32, P, i64,
                                     f32, P, P]
     L.bsa_mask_workspace_bytes.argtypes = [i32, i32, i32]
@@ -71,7 +73,7 @@ def lib():
     L.bsa_last_error.restype = ctypes.c_char_p
     L.bsa_check_device_error.argtypes = [P]
     L.bsa_selftest_wait_timeout.argtypes = [ctypes.c_uint64, P]
-    for name in ["stem_score", "stem_score_group", "bsa_prefill_group", "stem_score_noalloc", "stem_select", "bsa_prefill", "bsa_prefill_paged", "bsa_check_device_error",
+    for name in ["stem_score", "stem_score_group", "bsa_prefill_group", "bsa_prefill_skip", "stem_score_noalloc", "stem_select", "bsa_prefill", "bsa_prefill_paged", "bsa_check_device_error",
                  "bsa_selftest_wait_timeout", "bsa_mask_to_lists", "bsa_prefill_mask", "bsa_validate_lists"]:
         getattr(L, name).restype = ctypes.c_int
     _lib = L
@@ -219,6 +221,26 @@ def bsa_prefill(q, k, v, block: int, row_ptr, col_idx, softmax_scale: float = 0.
     st = lib().bsa_prefill(tensor_arg(q, q_scale), tensor_arg(k, k_scale), tensor_arg(v, v_scale), tensor_arg(out),
                            B, N, Hq, Hkv, d, block, _ptr(row_ptr), row_ptr.shape[-1], _ptr(col_idx),
                            col_idx.shape[-1], float(softmax_scale), _ptr(lse), _stream(q))
+    _check(st)
+    return (out, lse) if return_lse else out
+
+
+def bsa_prefill_skip(q, k, v, block: int, row_ptr, col_idx, skip_lambda: float, softmax_scale: float = 0.0,
+                     out=None, lse=None, return_lse: bool = False, q_scale=1.0, k_scale=1.0, v_scale=1.0,
+                     skip_stats=None):
+    """bsa_prefill with the threshold skip: a row drops a kept block whose max trails its running
+    max by more than ln(skip_lambda) (0 drops nothing).  skip_stats: optional int64 device tensor
+    of 4 counters (see bsa.h), incremented by the call."""
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    if out is None:
+        out = torch.empty(B, N, Hq, d, dtype=torch.bfloat16, device=q.device)
+    if return_lse and lse is None:
+        lse = torch.empty(B, Hq, N, dtype=torch.float32, device=q.device)
+    st = lib().bsa_prefill_skip(tensor_arg(q, q_scale), tensor_arg(k, k_scale), tensor_arg(v, v_scale),
+                                tensor_arg(out), B, N, Hq, Hkv, d, block, _ptr(row_ptr), row_ptr.shape[-1],
+                                _ptr(col_idx), col_idx.shape[-1], float(softmax_scale), float(skip_lambda),
+                                _ptr(lse), _ptr(skip_stats), _stream(q))
     _check(st)
     return (out, lse) if return_lse else out
 

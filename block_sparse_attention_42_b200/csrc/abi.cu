@@ -206,7 +206,8 @@ bsa_status_t prefill_launch(const bsa_tensor_t& q, const bsa_tensor_t& k, const 
                             const bsa_tensor_t& out, int32_t B, int32_t N, int32_t Hq, int32_t Hkv, int32_t d,
                             int32_t block, const int32_t* row_ptr, int32_t row_ptr_stride, int32_t row_ptr_hstride,
                             int32_t allow_empty, const int32_t* col_idx, int64_t max_k, float softmax_scale,
-                            float* lse, cudaStream_t stream, bool group = false) {
+                            float* lse, cudaStream_t stream, bool group = false, double skip_lambda = 0.0,
+                            unsigned long long* skip_stats = nullptr) {
     bsa_status_t st;
     const int nb = (N + block - 1) / block;
     bsa_status_t est;
@@ -247,6 +248,9 @@ bsa_status_t prefill_launch(const bsa_tensor_t& q, const bsa_tensor_t& k, const 
     a.lse_stride = N;
     a.err = err;
     a.list_per_group = group ? 1 : 0;
+    a.skip_on = skip_lambda > 0.0 ? 1 : 0;
+    a.skip_log2 = skip_lambda > 0.0 ? static_cast<float>(std::log2(skip_lambda)) : 0.f;
+    a.skip_stats = skip_stats;
     // Group-shared lists: the GQA-packed kernel where it applies (BSA_ATTN_VARIANT still picks a
     // per-head kernel for cross-checks), else the per-head kernels on the shared lists.
     const char* var = std::getenv("BSA_ATTN_VARIANT");
@@ -490,6 +494,30 @@ bsa_status_t bsa_prefill(bsa_tensor_t q, bsa_tensor_t k, bsa_tensor_t v, bsa_ten
     if (row_ptr_stride < nb + 1) return fail(BSA_ERR_INVALID_ARG, "row_ptr_stride must be >= nb + 1");
     return prefill_launch(q, k, v, out, B, N, Hq, Hkv, d, block, row_ptr, row_ptr_stride, 0, 0, col_idx, max_k,
                           softmax_scale, lse, stream);
+}
+
+bsa_status_t bsa_prefill_skip(bsa_tensor_t q, bsa_tensor_t k, bsa_tensor_t v, bsa_tensor_t out, int32_t B,
+                              int32_t N, int32_t Hq, int32_t Hkv, int32_t d, int32_t block, const int32_t* row_ptr,
+                              int32_t row_ptr_stride, const int32_t* col_idx, int64_t max_k, float softmax_scale,
+                              double skip_lambda, float* lse, unsigned long long* skip_stats,
+                              cudaStream_t stream) {
+    NvtxRange nvtx_range("bsa_prefill_skip");
+    bsa_status_t st;
+    if ((st = prefill_checks(q, k, v, out, B, N, Hq, Hkv, d, block, row_ptr, col_idx, max_k))) return st;
+    const int nb = (N + block - 1) / block;
+    if (row_ptr_stride < nb + 1) return fail(BSA_ERR_INVALID_ARG, "row_ptr_stride must be >= nb + 1");
+    if (!(skip_lambda >= 0.0 && skip_lambda < 1.0))
+        return fail(BSA_ERR_INVALID_ARG, "skip_lambda must be in [0, 1)");
+    if (skip_lambda > 0.0 && q.dtype == BSA_BF16 && d == 128 && block == 128)
+        return fail(BSA_ERR_UNSUPPORTED, "the threshold skip runs FP8, or BF16 with head_dim 64 or block 64");
+    const char* var = std::getenv("BSA_ATTN_VARIANT");
+    if (skip_lambda > 0.0 && var && std::strcmp(var, "ws3") != 0)
+        return fail(BSA_ERR_UNSUPPORTED, "the threshold skip runs in the default attention kernel only");
+    if (skip_stats && (reinterpret_cast<uintptr_t>(skip_stats) & 7u))
+        return fail(BSA_ERR_INVALID_ARG, "skip_stats must be 8-byte aligned");
+    // lambda = 0 runs the plain kernel; its statistics are then all zero and left untouched
+    return prefill_launch(q, k, v, out, B, N, Hq, Hkv, d, block, row_ptr, row_ptr_stride, 0, 0, col_idx, max_k,
+                          softmax_scale, lse, stream, false, skip_lambda, skip_stats);
 }
 
 bsa_status_t bsa_prefill_group(bsa_tensor_t q, bsa_tensor_t k, bsa_tensor_t v, bsa_tensor_t out, int32_t B,

@@ -77,11 +77,14 @@ struct Bars3 {
     uint64_t p_full[2], o_done[2];
     uint32_t tmem_slot;
     int abort_flag;
+    // Threshold skip: need[g % NP] == g + 1 when some row of block g kept it, so its PV runs.
+    int need[2];
     int lst[kListChunk3];
 };
 static_assert(sizeof(Bars3) <= 2048, "barrier region");
 
-template <bool FP8, int D, int BN, bool PAGED>
+// SKIP: the threshold-skip instantiation (bsa_prefill_skip); the default one has none of its code.
+template <bool FP8, int D, int BN, bool PAGED, bool SKIP>
 __global__ void __launch_bounds__(kThreads3, 2)
     attn_ws3_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                     const __grid_constant__ CUtensorMap tv, const AttnArgs a, int total_tiles) {
@@ -205,6 +208,7 @@ __global__ void __launch_bounds__(kThreads3, 2)
             const uint32_t aQ = smem_u32(smem + C::OFF_Q);
             const uint32_t aP = smem_u32(smem + C::OFF_P);
             uint32_t rbase = 0, qc = 0, pc = 0, sf = 0;
+            unsigned long long n_pv_skipped = 0;  // threshold skip: products not issued
             bool ok = true, first_s = true;
             TileIter it;
             it.init(0, blockIdx.x, gridDim.x, total_tiles);
@@ -239,13 +243,17 @@ __global__ void __launch_bounds__(kThreads3, 2)
             auto mma_pv = [&](uint32_t r, bool accumulate) -> bool {
                 const uint32_t pb = pc % C::NP;
                 if (!mbar_wait(&bars->p_full[pb], (pc / C::NP) & 1, abort_flag, a.err)) return false;
+                // With the threshold skip, a block that every row skipped has P = 0: no product.
+                const bool run = !SKIP || *reinterpret_cast<volatile int*>(&bars->need[pb]) ==
+                                              static_cast<int>(pc + 1);
+                if (SKIP) n_pv_skipped += run ? 0 : 1;
                 ++pc;
                 const int st = r % C::NS;
                 if (!mbar_wait(&bars->kv_full[st], (r / C::NS) & 1, abort_flag, a.err)) return false;
                 tc_fence_after();
                 const uint32_t aV = smem_u32(smem + C::OFF_RING + st * C::KV_BYTES);
 #pragma unroll
-                for (int kk = 0; kk < C::KSTEPS_O; ++kk) {
+                for (int kk = 0; kk < (run ? C::KSTEPS_O : 0); ++kk) {
                     const uint32_t byte = kk * 32, pan = byte / 128, within = byte % 128;
                     const uint64_t da = smem_desc_sw128(aP + pb * C::P_TILE + pan * kBM3 * 128 + within, 16, 1024);
                     const uint64_t db = smem_desc_sw128(aV + kk * C::ROWS_PER_KSTEP * 128, BN * 128, 1024);
@@ -276,6 +284,10 @@ __global__ void __launch_bounds__(kThreads3, 2)
                 rbase += 2 * n;
                 it.next(a);
             }
+            if (SKIP && a.skip_stats != nullptr) {
+                atomicAdd(a.skip_stats + 2, static_cast<unsigned long long>(pc));
+                atomicAdd(a.skip_stats + 3, n_pv_skipped);
+            }
             tc_commit(&bars->drain);
             volatile int no_abort = 0;
             mbar_wait(&bars->drain, 0, &no_abort, a.err);
@@ -301,6 +313,7 @@ __global__ void __launch_bounds__(kThreads3, 2)
             return __all_sync(0xFFFFFFFFu, w);
         };
         const float sl2 = a.scale_log2;
+        uint32_t n_vis = 0, n_skipped = 0;  // threshold skip: row-blocks of real rows, and skipped
         bool ok = true;
         TileIter it;
         it.init(0, blockIdx.x, gridDim.x, total_tiles);
@@ -308,6 +321,7 @@ __global__ void __launch_bounds__(kThreads3, 2)
         while (ok && it.active) {
             const Tile T = it.T;
             float m_used = -INFINITY, l_run = 0.f;
+            float m_true = -INFINITY;  // exact running max (log2 units), for the threshold skip
             int j_next = list_entry(a, T, 0);
             for (int k = 0; k < T.n_list; ++k) {
                 const int j = j_next;
@@ -365,17 +379,30 @@ __global__ void __launch_bounds__(kThreads3, 2)
                     mask_max(0);
                 }
                 const float mx = max3f(max3f(m8[0], m8[1], m8[2]), max3f(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
-                const float m_blk = mx * sl2;
+                float m_blk = mx * sl2;
+                // Threshold skip ([BLASST] §2.1): the row drops this block when its max trails the
+                // running max by more than log2(lambda); the block then adds nothing (P = 0).
+                bool skip = false;
+                if constexpr (SKIP) {
+                    skip = m_blk - m_true < a.skip_log2;
+                    m_true = fmaxf(m_true, m_blk);
+                    if (skip) m_blk = -INFINITY;
+                    if (row < a.block && T.i * a.block + row < T.n_tok) {
+                        ++n_vis;
+                        n_skipped += skip ? 1 : 0;
+                    }
+                }
+                const bool warp_skip = SKIP && __all_sync(0xFFFFFFFFu, skip);
                 float m_new = m_used;
                 if (m_blk > m_used + kRescale3<FP8>) m_new = m_blk;
                 const float alpha = (m_new == m_used) ? 1.f : fast_exp2(m_used - m_new);
-                const float mref = (m_new == -INFINITY) ? 0.f : m_new - kPScale3<FP8>;
-                // P = exp2(S * sl2 - mref) in place, four packed partial sums.
+                const float mref = skip ? INFINITY : ((m_new == -INFINITY) ? 0.f : m_new - kPScale3<FP8>);
+                // P = exp2(S * sl2 - mref) in place, four packed partial sums (a skipped row: 0).
                 const uint64_t sl2x2 = pack_f32x2(sl2, sl2);
                 const uint64_t negm = pack_f32x2(-mref, -mref);
                 uint64_t sum4[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-                for (int e = 0; e < BN; e += 2) {
+                for (int e = 0; e < (warp_skip ? 0 : BN); e += 2) {
                     const uint64_t x = fma_f32x2(pack_f32x2(__uint_as_float(rr[e]), __uint_as_float(rr[e + 1])),
                                                  sl2x2, negm);
                     float x0, x1;
@@ -394,6 +421,7 @@ __global__ void __launch_bounds__(kThreads3, 2)
                     tc_fence_after();
                 }
                 uint8_t* sPg = sP + (g % C::NP) * C::P_TILE;
+                if (SKIP && !warp_skip && lane == 0) bars->need[g % C::NP] = static_cast<int>(g + 1);
                 // P -> shared memory in the 128-byte-swizzled K-major layout of the PV A operand.
                 if constexpr (FP8) {
 #pragma unroll
@@ -402,8 +430,9 @@ __global__ void __launch_bounds__(kThreads3, 2)
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
                             const int e = unit * 16 + q * 4;
-                            w4[q] = pack_e4m3x4(__uint_as_float(rr[e]), __uint_as_float(rr[e + 1]),
-                                                __uint_as_float(rr[e + 2]), __uint_as_float(rr[e + 3]));
+                            w4[q] = warp_skip ? 0u
+                                              : pack_e4m3x4(__uint_as_float(rr[e]), __uint_as_float(rr[e + 1]),
+                                                            __uint_as_float(rr[e + 2]), __uint_as_float(rr[e + 3]));
                         }
                         const int pan = unit / 8, cc = unit % 8;
                         *reinterpret_cast<uint4*>(sPg + pan * kBM3 * 128 + row * 128 + ((cc ^ (row & 7)) * 16)) =
@@ -415,7 +444,9 @@ __global__ void __launch_bounds__(kThreads3, 2)
                         uint32_t w4[4];
 #pragma unroll
                         for (int q = 0; q < 4; ++q)
-                            w4[q] = pack_bf16x2(__uint_as_float(rr[unit * 8 + 2 * q]), __uint_as_float(rr[unit * 8 + 2 * q + 1]));
+                            w4[q] = warp_skip ? 0u
+                                              : pack_bf16x2(__uint_as_float(rr[unit * 8 + 2 * q]),
+                                                            __uint_as_float(rr[unit * 8 + 2 * q + 1]));
                         const int pan = unit / 8, cc = unit % 8;
                         *reinterpret_cast<uint4*>(sPg + pan * kBM3 * 128 + row * 128 + ((cc ^ (row & 7)) * 16)) =
                             make_uint4(w4[0], w4[1], w4[2], w4[3]);
@@ -492,6 +523,17 @@ __global__ void __launch_bounds__(kThreads3, 2)
             tc_fence_before();
             it.next(a);
         }
+        if (SKIP && a.skip_stats != nullptr) {
+            unsigned long long v0 = n_vis, v1 = n_skipped;
+            for (int o = 16; o > 0; o >>= 1) {
+                v0 += __shfl_xor_sync(0xFFFFFFFFu, v0, o);
+                v1 += __shfl_xor_sync(0xFFFFFFFFu, v1, o);
+            }
+            if (lane == 0) {
+                atomicAdd(a.skip_stats + 0, v0);
+                atomicAdd(a.skip_stats + 1, v1);
+            }
+        }
         tc_fence_before();
         mbar_arrive(&bars->tmem_free);
         return;
@@ -502,7 +544,7 @@ template <bool FP8, int D, int BN, bool PAGED>
 cudaError_t launch_ws3_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const AttnArgs& a,
                          cudaStream_t s) {
     using C = Cfg3<FP8, D, BN>;
-    auto kern = attn_ws3_kernel<FP8, D, BN, PAGED>;
+    auto kern = a.skip_on ? attn_ws3_kernel<FP8, D, BN, PAGED, true> : attn_ws3_kernel<FP8, D, BN, PAGED, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 148;

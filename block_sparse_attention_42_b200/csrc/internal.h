@@ -72,6 +72,10 @@ struct AttnArgs {
     const int32_t* page_table;   // paged only
     int max_pages, page_size, num_pages;
     float scale_log2;            // softmax scale * log2(e) (* q_scale * k_scale for FP8)
+    int skip_on;                 // 1: skip a block for a row whose block max trails its running max
+    float skip_log2;             //    by more than log2(lambda) = skip_log2 (threshold skip)
+    unsigned long long* skip_stats;  // nullable [4]: row-blocks visited, row-blocks skipped,
+                                     // tile-blocks, tile-blocks whose P.V product was skipped
     float out_scale;             // multiplies the normalised output (v_scale for FP8)
     void* out;
     int64_t osb, ost, osh;       // out element strides

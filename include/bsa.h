@@ -124,6 +124,29 @@ bsa_status_t bsa_prefill(bsa_tensor_t q, bsa_tensor_t k, bsa_tensor_t v, bsa_ten
                          const int32_t* row_ptr, int32_t row_ptr_stride, const int32_t* col_idx,
                          int64_t max_k, float softmax_scale, float* lse, cudaStream_t stream);
 
+/* bsa_prefill with a threshold skip on top of the lists ["BLASST: Dynamic BLocked Attention
+ * Sparsity via Softmax Thresholding" (gist.science), §2.1: skip a block whose local maximum
+ * trails the running maximum by more than ln(lambda)].  For each query row the kept blocks are
+ * visited in list order with an exact running maximum m of the scaled scores seen so far; a
+ * block whose largest scaled score over the row's allowed keys is below m + ln(skip_lambda) is
+ * skipped for that row (it contributes nothing; the output is the softmax over the other
+ * blocks' keys).  A warp whose 32 rows all skip a block skips its exponentials, and when every
+ * row of a query block skips it the P.V product is not issued.  skip_lambda in [0, 1); 0 skips
+ * nothing and computes exactly what bsa_prefill computes.  Runs FP8 (d 128, block 128), or BF16
+ * with head_dim 64 or block 64 (BSA_ERR_UNSUPPORTED otherwise); arguments, outputs and errors
+ * otherwise as in bsa_prefill.  The decisions are taken on fp32 scores, so a block whose max
+ * trails by almost exactly ln(skip_lambda) may be decided either way.
+ * skip_stats (nullable, device, 8-byte aligned, four uint64 the caller zeroes) is incremented by:
+ * [0] (row, kept block) pairs visited, over the rows that are tokens of the sequence; [1] how
+ * many of them were skipped; [2] (query block, kept block) pairs; [3] how many of those had
+ * every row skip, so that no P.V product was issued.  With skip_lambda = 0 it is not touched. */
+bsa_status_t bsa_prefill_skip(bsa_tensor_t q, bsa_tensor_t k, bsa_tensor_t v, bsa_tensor_t out,
+                              int32_t B, int32_t N, int32_t Hq, int32_t Hkv, int32_t d,
+                              int32_t block, const int32_t* row_ptr, int32_t row_ptr_stride,
+                              const int32_t* col_idx, int64_t max_k, float softmax_scale,
+                              double skip_lambda, float* lse, unsigned long long* skip_stats,
+                              cudaStream_t stream);
+
 /* Group-shared selection with GQA-packed attention.  The pages select per query head and say
  * nothing about grouped-query attention.  This extension gives the G = Hq / Hkv query heads of
  * a KV-head group one kept-block list, so that the heads sharing a list can share every K/V
