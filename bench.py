@@ -54,6 +54,7 @@ def parse():
                    help="skip the density, length and paged-varlen sweeps of bsa_prefill")
     p.add_argument("--sweep-reps", type=int, default=3, help="timed calls per sweep point")
     p.add_argument("--no-skip", action="store_true", help="skip the threshold-skip (bsa_prefill_skip) measurement")
+    p.add_argument("--no-fused", action="store_true", help="skip the stem_score_select measurement")
     p.add_argument("--no-group", action="store_true",
                    help="skip the group-shared selection + GQA-packed attention measurement")
     return p.parse_args()
@@ -559,6 +560,27 @@ def run_ours(args, rank, world, device):
                         "per_head_bsa_prefill_ms": res["attn_ms"], "reps": reps}
         del g_scores, g_ws, g_rp, g_ci, g_out
 
+    # Score + select in one call without the score matrix: same lists, timed like select_ms.
+    if not args.no_fused and rank == 0:
+        f_ws = torch.empty(bsa.bsa_score_select_workspace_bytes(B, Hq, Hkv, N, w.block, D), dtype=torch.uint8,
+                           device=device)
+        f_rp = torch.empty(B, nb + 1, dtype=torch.int32, device=device)
+        f_ci = torch.empty(B, Hq, kstar, dtype=torch.int32, device=device)
+
+        def fused():
+            bsa.stem_score_select(q, k, v, w.block, w.density, 0.5, row_ptr=f_rp, col_idx=f_ci, max_k=kstar,
+                                  workspace=f_ws, **scale_kw)
+
+        f_ms = _time_calls(fused, max(3, min(args.steps, 10)), stream)
+        bsa.bsa_check_device_error(device)
+        same = bool(torch.equal(f_rp, row_ptr) and torch.equal(f_ci, col_idx))
+        res["fused_select"] = {"what": "stem_score_select: pool, budget, then per chunk of KV-head groups the score "
+                                       "GEMM into an L2-sized scratch and the top-k from it; no score matrix",
+                               "ms": f_ms, "unfused_select_ms": res["select_ms"], "lists_equal_unfused": same,
+                               "workspace_bytes": f_ws.numel(),
+                               "unfused_bytes": scores.numel() * 4 + ws.numel()}
+        del f_ws, f_rp, f_ci
+
     # Threshold skip on top of the step's lists: speed and the kernel's own skip counters.
     if not args.no_skip and rank == 0 and (fp8 or D == 64 or w.block == 64):
         pts = []
@@ -811,6 +833,8 @@ def main():
             line["group_shared"] = res["group"]
         if "skip" in res:
             line["threshold_skip"] = res["skip"]
+        if "fused_select" in res:
+            line["fused_select"] = res["fused_select"]
         if "mask" in res:
             m = dict(res["mask"])
             m["mask_to_lists_roofline"] = {"bound": "hbm", "achieved": m.pop("mask_to_lists_gbs"),

@@ -26,7 +26,7 @@ EXPORTS = ["bsa_tpd_budget", "bsa_score_workspace_bytes", "stem_score", "stem_se
            "bsa_prefill_paged", "bsa_last_error", "bsa_check_device_error", "stem_score_noalloc",
            "bsa_selftest_wait_timeout", "bsa_mask_workspace_bytes", "bsa_mask_to_lists", "bsa_prefill_mask",
            "bsa_validate_lists", "bsa_score_group_workspace_bytes", "stem_score_group", "bsa_prefill_group",
-           "bsa_prefill_skip"]
+           "bsa_prefill_skip", "bsa_score_select_workspace_bytes", "stem_score_select"]
 
 
 class BsaError(RuntimeError):
@@ -56,6 +56,10 @@ def lib():
     L.bsa_score_workspace_bytes.restype = ctypes.c_size_t
     L.stem_score.argtypes = [T, T, T, i32, i32, i32, i32, i32, i32, i32, f32, P, i32, P, ctypes.c_size_t, P]
     L.stem_score_group.argtypes = L.stem_score.argtypes
+    L.stem_score_select.argtypes = [T, T, T, i32, i32, i32, i32, i32, i32, i32, f32, f64, f64, P, P, i64, P,
+                                    ctypes.c_size_t, P]
+    L.bsa_score_select_workspace_bytes.argtypes = [i32, i32, i32, i32, i32, i32]
+    L.bsa_score_select_workspace_bytes.restype = ctypes.c_size_t
     L.bsa_score_group_workspace_bytes.argtypes = [i32, i32, i32, i32, i32]
     L.bsa_score_group_workspace_bytes.restype = ctypes.c_size_t
     L.stem_score_noalloc.argtypes = [T, T, T, i32, i32, i32, i32, i32, i32, i32, f32, P, i32, P]
@@ -73,7 +77,7 @@ def lib():
     L.bsa_last_error.restype = ctypes.c_char_p
     L.bsa_check_device_error.argtypes = [P]
     L.bsa_selftest_wait_timeout.argtypes = [ctypes.c_uint64, P]
-    for name in ["stem_score", "stem_score_group", "bsa_prefill_group", "bsa_prefill_skip", "stem_score_noalloc", "stem_select", "bsa_prefill", "bsa_prefill_paged", "bsa_check_device_error",
+    for name in ["stem_score", "stem_score_select", "stem_score_group", "bsa_prefill_group", "bsa_prefill_skip", "stem_score_noalloc", "stem_select", "bsa_prefill", "bsa_prefill_paged", "bsa_check_device_error",
                  "bsa_selftest_wait_timeout", "bsa_mask_to_lists", "bsa_prefill_mask", "bsa_validate_lists"]:
         getattr(L, name).restype = ctypes.c_int
     _lib = L
@@ -174,6 +178,34 @@ def stem_score_group(q, k, v, block: int, metric: int = BSA_METRIC_OAM, softmax_
                                 workspace.numel(), _stream(q))
     _check(st)
     return scores
+
+
+def bsa_score_select_workspace_bytes(B, Hq, Hkv, N, block, d) -> int:
+    return int(lib().bsa_score_select_workspace_bytes(B, Hq, Hkv, N, block, d))
+
+
+def stem_score_select(q, k, v, block: int, density: float, tpd_decay: float = 0.5, metric: int = BSA_METRIC_OAM,
+                      softmax_scale: float = 0.0, row_ptr=None, col_idx=None, max_k: int | None = None,
+                      workspace=None, q_scale=1.0, k_scale=1.0, v_scale=1.0):
+    """Score + TPD select without the score matrix: (row_ptr [B, nb+1], col_idx [B, Hq, max_k])."""
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    nb = (N + block - 1) // block
+    if max_k is None:
+        max_k = tpd_kstar(nb, density, tpd_decay)
+    if row_ptr is None:
+        row_ptr = torch.empty(B, nb + 1, dtype=torch.int32, device=q.device)
+    if col_idx is None:
+        col_idx = torch.empty(B, Hq, max_k, dtype=torch.int32, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(bsa_score_select_workspace_bytes(B, Hq, Hkv, N, block, d), dtype=torch.uint8,
+                                device=q.device)
+    st = lib().stem_score_select(tensor_arg(q, q_scale), tensor_arg(k, k_scale), tensor_arg(v, v_scale), B, N, Hq,
+                                 Hkv, d, block, metric, float(softmax_scale), float(density), float(tpd_decay),
+                                 _ptr(row_ptr), _ptr(col_idx), int(max_k), _ptr(workspace), workspace.numel(),
+                                 _stream(q))
+    _check(st)
+    return row_ptr, col_idx
 
 
 def stem_score_noalloc(q, k, v, block: int, metric: int = BSA_METRIC_OAM, softmax_scale: float = 0.0,

@@ -435,6 +435,19 @@ bsa_status_t score_common(bool group, const bsa_tensor_t& q, const bsa_tensor_t&
     return BSA_OK;
 }
 
+// stem_score_select: the score matrix of one chunk of KV-head groups of one sequence at a time,
+// so that at most kScoreChunkBytes of it exist at once (L2-resident), consumed by the top-k.
+constexpr size_t kScoreChunkBytes = size_t(64) << 20;
+
+int score_select_groups(int32_t Hq, int32_t Hkv, int nb) {
+    const size_t per_group = sizeof(float) * size_t(Hq / Hkv) * nb * nb;
+    int cg = static_cast<int>(kScoreChunkBytes / per_group);
+    if (cg < 1) cg = 1;
+    if (cg > Hkv) cg = Hkv;
+    while (Hkv % cg) --cg;
+    return cg;
+}
+
 }  // namespace
 }  // namespace bsa
 
@@ -454,6 +467,95 @@ bsa_status_t stem_score_group(bsa_tensor_t q, bsa_tensor_t k, bsa_tensor_t v, in
     NvtxRange nvtx_range("stem_score_group");
     return score_common(true, q, k, v, B, N, Hq, Hkv, d, block, metric, softmax_scale, scores, nb_stride, ws,
                         ws_bytes, stream);
+}
+
+size_t bsa_score_select_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int32_t N, int32_t block,
+                                        int32_t d) {
+    if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || N < 1 || block < 1 || d < 1) return 0;
+    const int nb = (N + block - 1) / block;
+    const int cg = score_select_groups(Hq, Hkv, nb);
+    return bsa_score_workspace_bytes(B, Hq, Hkv, nb, d) +
+           align256(sizeof(float) * size_t(cg) * (Hq / Hkv) * nb * nb);
+}
+
+bsa_status_t stem_score_select(bsa_tensor_t q, bsa_tensor_t k, bsa_tensor_t v, int32_t B, int32_t N, int32_t Hq,
+                               int32_t Hkv, int32_t d, int32_t block, int32_t metric, float softmax_scale,
+                               double density, double tpd_decay, int32_t* row_ptr, int32_t* col_idx, int64_t max_k,
+                               void* ws, size_t ws_bytes, cudaStream_t stream) {
+    NvtxRange nvtx_range("stem_score_select");
+    bsa_status_t st;
+    if ((st = check_tensor(q, "q", B > 1)) || (st = check_tensor(k, "k", B > 1)) || (st = check_tensor(v, "v", B > 1)))
+        return st;
+    if (q.dtype != k.dtype || q.dtype != v.dtype) return fail(BSA_ERR_INVALID_ARG, "q, k and v must share a dtype");
+    if (B < 1 || N < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv)
+        return fail(BSA_ERR_INVALID_ARG, "bad sizes (B=%d N=%d Hq=%d Hkv=%d)", B, N, Hq, Hkv);
+    if (B > kMaxBatch) return fail(BSA_ERR_UNSUPPORTED, "B must be in [1, %d]", kMaxBatch);
+    if (d != 64 && d != 128) return fail(BSA_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
+    if (block != 64 && block != 128) return fail(BSA_ERR_UNSUPPORTED, "block must be 64 or 128");
+    if (metric < BSA_METRIC_OAM || metric > BSA_METRIC_OAM_MUL) return fail(BSA_ERR_INVALID_ARG, "unknown metric");
+    const int nb = (N + block - 1) / block;
+    if (nb > kMaxBlocks) return fail(BSA_ERR_UNSUPPORTED, "at most %d blocks per sequence", kMaxBlocks);
+    if (!row_ptr || !col_idx) return fail(BSA_ERR_INVALID_ARG, "row_ptr/col_idx are null");
+    if (!(density > 0.0 && density <= 1.0)) return fail(BSA_ERR_INVALID_ARG, "density must be in (0, 1]");
+    if (!(tpd_decay == 0.0 || tpd_decay == 0.5)) return fail(BSA_ERR_UNSUPPORTED, "tpd_decay must be 0 or 0.5");
+    const int64_t kstar = tpd_kstar(nb, density);
+    if (kstar > max_k)
+        return fail(BSA_ERR_INVALID_ARG, "max_k=%lld is below the budget %lld", (long long)max_k, (long long)kstar);
+    const size_t need = bsa_score_select_workspace_bytes(B, Hq, Hkv, N, block, d);
+    if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u))
+        return fail(BSA_ERR_WORKSPACE, "workspace must be >= %zu bytes and 256-byte aligned", need);
+    bsa_status_t est;
+    unsigned* err = device_error_word(&est);
+    if (err == nullptr) return est;
+    // Workspace: the pooled means as in stem_score, then the score chunk.
+    const size_t qbytes = align256(sizeof(float) * size_t(B) * Hq * nb * d);
+    const size_t kbytes = align256(sizeof(float) * size_t(B) * Hkv * nb * d);
+    const size_t vbytes = align256(sizeof(float) * size_t(B) * Hkv * nb);
+    char* w = static_cast<char*>(ws);
+    float* qhi = reinterpret_cast<float*>(w);
+    float* qlo = reinterpret_cast<float*>(w + qbytes);
+    float* khi = reinterpret_cast<float*>(w + 2 * qbytes);
+    float* klo = reinterpret_cast<float*>(w + 2 * qbytes + kbytes);
+    float* vbar = reinterpret_cast<float*>(w + 2 * qbytes + 2 * kbytes);
+    float* chunk = reinterpret_cast<float*>(w + 2 * qbytes + 2 * kbytes + vbytes);
+    const float tau = softmax_scale > 0.f ? softmax_scale : 1.f / std::sqrt(static_cast<float>(d));
+    const int dt = q.dtype == BSA_BF16 ? 0 : (q.dtype == BSA_FP8_E4M3 ? 1 : 2);
+    cudaError_t e =
+        launch_pool(dt, targ(q), targ(k), targ(v), B, N, Hq, Hkv, d, block, qhi, qlo, khi, klo, vbar, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "pool launch");
+    SelectSeqs all;
+    all.B = B;
+    for (int b = 0; b < B; ++b) {
+        all.nb[b] = nb;
+        all.kstar[b] = kstar;
+    }
+    e = launch_tpd_budget(all, nb, tpd_decay == 0.5, row_ptr, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "budget launch");
+    SelectSeqs one;
+    one.B = 1;
+    one.nb[0] = nb;
+    one.kstar[0] = kstar;
+    const int G = Hq / Hkv, cg = score_select_groups(Hq, Hkv, nb);
+    const int64_t hs = int64_t(nb) * d;  // floats per head of a pooled tensor
+    for (int b = 0; b < B; ++b) {
+        for (int hk0 = 0; hk0 < Hkv; hk0 += cg) {
+            const int h0 = hk0 * G;
+            CUtensorMap mqh, mql, mkh, mkl;
+            const int64_t qo = (int64_t(b) * Hq + h0) * hs, ko = (int64_t(b) * Hkv + hk0) * hs;
+            if ((st = make_map(&mqh, qhi + qo, 4, d, nb, cg * G, 1, d, hs, hs * Hq, 128, "qhi")) ||
+                (st = make_map(&mql, qlo + qo, 4, d, nb, cg * G, 1, d, hs, hs * Hq, 128, "qlo")) ||
+                (st = make_map(&mkh, khi + ko, 4, d, nb, cg, 1, d, hs, hs * Hkv, 128, "khi")) ||
+                (st = make_map(&mkl, klo + ko, 4, d, nb, cg, 1, d, hs, hs * Hkv, 128, "klo")))
+                return st;
+            e = launch_score_tc(mqh, mql, mkh, mkl, vbar + (int64_t(b) * Hkv + hk0) * nb, 1, cg * G, cg, nb, d, tau,
+                                metric, chunk, nb, err, stream);
+            if (e != cudaSuccess) return cuda_fail(e, "score launch");
+            e = launch_select_rows(chunk, one, cg * G, nb, row_ptr + int64_t(b) * (nb + 1),
+                                   col_idx + (int64_t(b) * Hq + h0) * max_k, max_k, stream);
+            if (e != cudaSuccess) return cuda_fail(e, "select launch");
+        }
+    }
+    return BSA_OK;
 }
 
 bsa_status_t stem_select(const float* scores, int32_t B, int32_t Hq, const int32_t* nb_per_seq, int32_t nb_stride,

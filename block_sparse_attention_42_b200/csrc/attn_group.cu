@@ -21,6 +21,11 @@
 //   warps 4-7   softmax of slot 0, warps 8-11 softmax of slot 1: one query row per thread (TMEM
 //               lane quadrant = warp % 4), as in the per-head kernels.
 // Per slot two P buffers: P(k) only waits for PV(k-2).
+// The two slots read the same blocks, so their S products land together and, left alone, their
+// exponential phases would run at the same time: the MUFU (16 ex2 per clock per SM) would be
+// shared while both exponentiate and idle while both do the rest of a block.  A token makes the
+// slots take turns at the exponentials, so one slot's exponentials overlap the other's loads,
+// max, P stores and rescale (measured at fp8-128k: 52.3 ms against 56.7 ms without it).
 // Tensor memory (512 columns): S slot 0 | S slot 1 | O slot 0 | O slot 1.
 #include <cuda_bf16.h>
 
@@ -71,6 +76,9 @@ struct CfgG {
 // E4M3: the running max moves only when the row max grew by more than 2^5, with P scaled by
 // 2^3, so P <= 2^8 fits E4M3 and values down to 2^-12 of the row max keep E4M3 precision.
 constexpr float kRescaleG = 5.f;
+// A slot waits at most this long for its turn, then goes on without it (the token only orders
+// the slots' exponentials; it is never needed for correctness).
+constexpr uint64_t kTurnLimitNs = 20000;
 constexpr float kPScaleG = 3.f;
 
 struct SlotBarsG {
@@ -83,6 +91,9 @@ struct BarsG {
     uint64_t q_full, q_empty;
     SlotBarsG sl[kSlotsG];
     uint64_t tmem_free;
+    // Exponential-phase token: slot s waits on turn[s] before its exponentials and hands the
+    // turn to the other slot after them, so the two slots' exponentials alternate.
+    uint64_t turn[kSlotsG];
     uint32_t tmem_slot;
     int abort_flag;
     int lst[kListChunkG];  // list entries staged by the producer warp
@@ -156,6 +167,8 @@ __global__ void __launch_bounds__(kThreadsG, 1)
             mbar_init(&B.drain, 1);
         }
         mbar_init(&bars->tmem_free, 256);
+        mbar_init(&bars->turn[0], 128);
+        mbar_init(&bars->turn[1], 128);
         bars->abort_flag = 0;
         fence_barrier_init();
         tma_prefetch_desc(&tq);
@@ -369,6 +382,9 @@ __global__ void __launch_bounds__(kThreadsG, 1)
     };
     const float sl2 = a.scale_log2;
     bool ok = true;
+    // Slot 0 takes the first turn: slot 1 hands it over once at the start.
+    if (slot == 1) mbar_arrive(&bars->turn[0]);
+    uint32_t turns = 0;
     UnitIter it;
     it.init(blockIdx.x, gridDim.x, total_units);
     it.next(a);
@@ -424,6 +440,13 @@ __global__ void __launch_bounds__(kThreadsG, 1)
             if (m_blk > m_used + kRescaleG) m_new = m_blk;
             const float alpha = (m_new == m_used) ? 1.f : fast_exp2(m_used - m_new);
             const float mref = (m_new == -INFINITY) ? 0.f : m_new - kPScaleG;
+            // Wait for this slot's turn (bounded: past the limit it goes on without it).
+            {
+                const uint64_t t0 = globaltimer_ns();
+                while (!mbar_try_wait(&bars->turn[slot], turns & 1))
+                    if (globaltimer_ns() - t0 > kTurnLimitNs) break;
+                ++turns;
+            }
             // P = exp2(S * sl2 - mref) in place, four packed partial sums.
             const uint64_t sl2x2 = pack_f32x2(sl2, sl2);
             const uint64_t negm = pack_f32x2(-mref, -mref);
@@ -439,6 +462,7 @@ __global__ void __launch_bounds__(kThreadsG, 1)
                 rr[e] = __float_as_uint(p0);
                 rr[e + 1] = __float_as_uint(p1);
             }
+            mbar_arrive(&bars->turn[slot ^ 1]);
             // The PV that last read this P buffer (block g - 2) must be complete.
             if (g >= static_cast<uint32_t>(C::NP)) {
                 if (!wait_pv(g - C::NP)) {

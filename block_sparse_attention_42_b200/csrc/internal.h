@@ -53,6 +53,12 @@ struct SelectSeqs {
 // a3 + a4: TPD budgets into row_ptr, then per-row top-k lists into col_idx.
 cudaError_t launch_select(const float* scores, const SelectSeqs& seqs, int Hq, int nb_stride, bool decay_half,
                           int32_t* row_ptr, int32_t* col_idx, int64_t max_k, cudaStream_t s);
+// The two halves of launch_select: the budget (row_ptr [B, nb_stride + 1]) and the per-row top-k
+// of scores [B, Hq, nb_stride, nb_stride] into col_idx [B, Hq, max_k] (row_ptr already written).
+cudaError_t launch_tpd_budget(const SelectSeqs& seqs, int nb_stride, bool decay_half, int32_t* row_ptr,
+                              cudaStream_t s);
+cudaError_t launch_select_rows(const float* scores, const SelectSeqs& seqs, int Hq, int nb_stride,
+                               const int32_t* row_ptr, int32_t* col_idx, int64_t max_k, cudaStream_t s);
 
 // a5: block-sparse prefill.
 struct AttnArgs {

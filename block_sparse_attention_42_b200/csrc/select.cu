@@ -328,17 +328,28 @@ cudaError_t launch_sel(const float* scores, const SelectSeqs& seqs, int Hq, int 
 
 }  // namespace
 
-cudaError_t launch_select(const float* scores, const SelectSeqs& seqs, int Hq, int nb_stride, bool decay_half,
-                          int32_t* row_ptr, int32_t* col_idx, int64_t max_k, cudaStream_t s) {
+cudaError_t launch_tpd_budget(const SelectSeqs& seqs, int nb_stride, bool decay_half, int32_t* row_ptr,
+                              cudaStream_t s) {
     tpd_budget_kernel<<<seqs.B, kBudgetThreads, 0, s>>>(seqs, decay_half ? 1 : 0, row_ptr, nb_stride);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+cudaError_t launch_select_rows(const float* scores, const SelectSeqs& seqs, int Hq, int nb_stride,
+                               const int32_t* row_ptr, int32_t* col_idx, int64_t max_k, cudaStream_t s) {
+    cudaError_t e;
     // One launch per row-length class, longest rows first: i in [1024, 2048), [512, 1024),
     // [256, 512), [0, 256).
     if ((e = launch_sel<64>(scores, seqs, Hq, nb_stride, row_ptr, col_idx, max_k, s)) != cudaSuccess) return e;
     if ((e = launch_sel<32>(scores, seqs, Hq, nb_stride, row_ptr, col_idx, max_k, s)) != cudaSuccess) return e;
     if ((e = launch_sel<16>(scores, seqs, Hq, nb_stride, row_ptr, col_idx, max_k, s)) != cudaSuccess) return e;
     return launch_sel<8>(scores, seqs, Hq, nb_stride, row_ptr, col_idx, max_k, s);
+}
+
+cudaError_t launch_select(const float* scores, const SelectSeqs& seqs, int Hq, int nb_stride, bool decay_half,
+                          int32_t* row_ptr, int32_t* col_idx, int64_t max_k, cudaStream_t s) {
+    cudaError_t e = launch_tpd_budget(seqs, nb_stride, decay_half, row_ptr, s);
+    if (e != cudaSuccess) return e;
+    return launch_select_rows(scores, seqs, Hq, nb_stride, row_ptr, col_idx, max_k, s);
 }
 
 }  // namespace bsa

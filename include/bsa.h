@@ -113,6 +113,25 @@ bsa_status_t stem_select(const float* scores, int32_t B, int32_t Hq, const int32
                          int32_t nb_stride, double density, double tpd_decay, int32_t* row_ptr,
                          int32_t* col_idx, int64_t max_k, cudaStream_t stream);
 
+/* Score and select in one call, without the score matrix [cn486 page, §二.2.1 Stem算子优化:
+ * budget generation and the selection sort are fused, with no large intermediates].  Computes
+ * exactly what stem_score followed by stem_select computes (the same lists, bit for bit: the
+ * same per-tile score products and the same per-row selection), for B sequences of N tokens
+ * (nb = ceil(N / block) blocks each), without a [B, Hq, nb, nb] score buffer.  The scores of one
+ * chunk of KV-head groups of one sequence exist at a time, in `ws` (at most 64 MiB of it, or one
+ * group when a group alone is larger), and are consumed by the top-k before the next chunk is
+ * scored.  Outputs: row_ptr [B, nb + 1] and col_idx [B, Hq, max_k] as stem_select writes them;
+ * max_k >= bsa_tpd_budget(nb, density, tpd_decay, NULL).  ws: at least
+ * bsa_score_select_workspace_bytes() bytes, 256-byte aligned.  Arguments and errors otherwise as
+ * in stem_score and stem_select; bsa_score_select_workspace_bytes returns 0 for invalid sizes. */
+size_t bsa_score_select_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int32_t N, int32_t block,
+                                        int32_t d);
+bsa_status_t stem_score_select(bsa_tensor_t q, bsa_tensor_t k, bsa_tensor_t v, int32_t B, int32_t N,
+                               int32_t Hq, int32_t Hkv, int32_t d, int32_t block, int32_t metric,
+                               float softmax_scale, double density, double tpd_decay,
+                               int32_t* row_ptr, int32_t* col_idx, int64_t max_k, void* ws,
+                               size_t ws_bytes, cudaStream_t stream);
+
 /* Block-sparse causal prefill.  q [B, N, Hq, d]; k, v [B, N, Hkv, d] (BF16, or FP8_E4M3 with
  * per-tensor scales); out [B, N, Hq, d] BF16.  For token t of head h the allowed keys are the
  * tokens s <= t whose block is in the list (row_ptr/col_idx as produced by stem_select, with
