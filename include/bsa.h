@@ -19,6 +19,16 @@
  *   bsa_mask_to_lists / bsa_prefill_mask
  *                the same attention with the selection given as a uint8 block mask per
  *                (sequence, query head), the form HPC-BSA takes it in [same page, §二.2.2].
+ *   stem_score_select
+ *                stem_score + stem_select in one call without the score matrix [same page,
+ *                §二.2.1: no large intermediates].
+ *   stem_score_group / bsa_prefill_group
+ *                one list per KV-head group shared by its query heads, and attention that loads
+ *                each kept K/V block once for two heads (an extension; the pages say nothing
+ *                about grouped-query attention).
+ *   bsa_prefill_skip
+ *                bsa_prefill with a threshold skip on top of the lists ["BLASST: Dynamic BLocked
+ *                Attention Sparsity via Softmax Thresholding", §2.1].
  *
  * Conventions shared by every call:
  *   - All pointers except those marked "host" are device pointers on the current device.
