@@ -66,6 +66,17 @@ __device__ __forceinline__ int list_entry(const AttnArgs& a, const Tile& T, int 
     return (j >= 0 && j <= T.i) ? j : -1;
 }
 
+// Entry n of the tile's list as stored (0 for n past the end, which no block uses), and the
+// range check of list_entry applied to such a value: the two halves of list_entry for a
+// caller that loads entries ahead of their use.
+__device__ __forceinline__ int list_entry_raw(const AttnArgs& a, const Tile& T, int n) {
+    if (n >= T.n_list) return 0;
+    const int64_t row = a.list_per_group ? static_cast<int64_t>(T.b) * a.Hkv + T.hk
+                                         : static_cast<int64_t>(T.b) * a.Hq + T.h;
+    return __ldg(a.col_idx + row * a.max_k + T.l_begin + n);
+}
+__device__ __forceinline__ int list_entry_check(const Tile& T, int j) { return (j >= 0 && j <= T.i) ? j : -1; }
+
 // The static tile sequence of one slot: tiles base + s, base + s + stride, ... that are
 // non-empty.  Every role walks the same sequence.
 struct TileIter {

@@ -322,10 +322,17 @@ __global__ void __launch_bounds__(kThreads3, 2)
             const Tile T = it.T;
             float m_used = -INFINITY, l_run = 0.f;
             float m_true = -INFINITY;  // exact running max (log2 units), for the threshold skip
-            int j_next = list_entry(a, T, 0);
+            // The tile's list, 32 entries per warp-wide load: lane e holds entry 32c + e of the
+            // current chunk c, and the next chunk is loaded a chunk ahead, so no block waits on
+            // a global load; block k's entry is a shuffle.
+            int jl = list_entry_raw(a, T, lane);
+            int jl_next = list_entry_raw(a, T, 32 + lane);
             for (int k = 0; k < T.n_list; ++k) {
-                const int j = j_next;
-                if (k + 1 < T.n_list) j_next = list_entry(a, T, k + 1);
+                if ((k & 31) == 0 && k > 0) {
+                    jl = jl_next;
+                    jl_next = list_entry_raw(a, T, k + 32 + lane);
+                }
+                const int j = list_entry_check(T, __shfl_sync(0xFFFFFFFFu, jl, k & 31));
                 bool w_ok = mbar_wait(&bars->s_full, scount & 1, abort_flag, a.err);
                 ++scount;
                 w_ok = __all_sync(0xFFFFFFFFu, w_ok);
@@ -395,7 +402,7 @@ __global__ void __launch_bounds__(kThreads3, 2)
                 const bool warp_skip = SKIP && __all_sync(0xFFFFFFFFu, skip);
                 float m_new = m_used;
                 if (m_blk > m_used + kRescale3<FP8>) m_new = m_blk;
-                const float alpha = (m_new == m_used) ? 1.f : fast_exp2(m_used - m_new);
+                const bool moved = m_new != m_used;
                 const float mref = skip ? INFINITY : ((m_new == -INFINITY) ? 0.f : m_new - kPScale3<FP8>);
                 // P = exp2(S * sl2 - mref) in place, four packed partial sums (a skipped row: 0).
                 const uint64_t sl2x2 = pack_f32x2(sl2, sl2);
@@ -453,9 +460,12 @@ __global__ void __launch_bounds__(kThreads3, 2)
                     }
                 }
                 fence_proxy_async_smem();
-                if (k > 0 && __any_sync(0xFFFFFFFFu, alpha != 1.f)) {
+                float alpha = 1.f;
+                if (k > 0 && __any_sync(0xFFFFFFFFu, moved)) {
                     // O *= alpha once PV(k-1) has finished accumulating into it, 64 TMEM columns at
-                    // a time (P is in shared memory, rr is free).
+                    // a time (P is in shared memory, rr is free).  (At k = 0 there is no O yet and
+                    // l_run is 0, so the factor is not needed.)
+                    if (moved) alpha = fast_exp2(m_used - m_new);
                     if (C::NP > 1) {
                         if (!wait_pv(g - 1)) {
                             ok = false;
