@@ -17,6 +17,8 @@
 namespace bsa {
 
 __device__ unsigned g_device_error;  // per-device error word (kDevErr* bits)
+constexpr int kTileCounters = 64;
+__device__ int g_tile_counter[kTileCounters];  // per-launch counters of the dynamic tile schedule
 
 namespace {
 
@@ -84,6 +86,41 @@ unsigned* device_error_word(bsa_status_t* st) {
     }
     *st = BSA_OK;
     return static_cast<unsigned*>(addr[dev]);
+}
+
+// A tile counter for one attention launch, zeroed on `stream` ahead of it.  Launches take the
+// per-device slots in turn, so two launches in flight share one only when 64 others were
+// issued between them.
+int* tile_counter(cudaStream_t stream, bsa_status_t* st) {
+    static std::mutex mu;
+    static void* base[64] = {};
+    static unsigned turn[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess || dev < 0 || dev >= 64) {
+        *st = cuda_fail(e, "cudaGetDevice");
+        return nullptr;
+    }
+    int* p = nullptr;
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        if (base[dev] == nullptr) {
+            e = cudaGetSymbolAddress(&base[dev], g_tile_counter);
+            if (e != cudaSuccess) {
+                base[dev] = nullptr;
+                *st = cuda_fail(e, "cudaGetSymbolAddress(tile counters)");
+                return nullptr;
+            }
+        }
+        p = static_cast<int*>(base[dev]) + (turn[dev]++ % kTileCounters);
+    }
+    e = cudaMemsetAsync(p, 0, sizeof(int), stream);
+    if (e != cudaSuccess) {
+        *st = cuda_fail(e, "cudaMemsetAsync(tile counter)");
+        return nullptr;
+    }
+    *st = BSA_OK;
+    return p;
 }
 
 // ---------------------------------------------------------------- TPD budget (host copy)
@@ -251,6 +288,7 @@ bsa_status_t prefill_launch(const bsa_tensor_t& q, const bsa_tensor_t& k, const 
     a.skip_on = skip_lambda > 0.0 ? 1 : 0;
     a.skip_log2 = skip_lambda > 0.0 ? static_cast<float>(std::log2(skip_lambda)) : 0.f;
     a.skip_stats = skip_stats;
+    if (!(a.tile_counter = tile_counter(stream, &est))) return est;
     // Group-shared lists: the GQA-packed kernel where it applies (BSA_ATTN_VARIANT still picks a
     // per-head kernel for cross-checks), else the per-head kernels on the shared lists.
     const char* var = std::getenv("BSA_ATTN_VARIANT");
@@ -818,6 +856,7 @@ bsa_status_t bsa_prefill_paged(bsa_tensor_t q, bsa_tensor_t out, const int32_t* 
     a.lse = lse;
     a.lse_stride = n_max;
     a.err = err;
+    if (!(a.tile_counter = tile_counter(stream, &est))) return est;
     cudaError_t e = launch_attn(fp8, true, tq, tk, tv, a, stream);
     if (e != cudaSuccess) return cuda_fail(e, "bsa_prefill_paged launch");
     return BSA_OK;

@@ -31,6 +31,7 @@ constexpr int kThreads3 = 192;
 constexpr int kSmem3Limit = 115712;  // two CTAs per SM
 constexpr int kMaxStages3 = 6;
 constexpr int kListChunk3 = 128;
+constexpr int kTileRing3 = 4;  // tile indices handed from the producer to the MMA and softmax warps
 
 template <bool FP8, int D, int BN>
 struct Cfg3 {
@@ -79,6 +80,11 @@ struct Bars3 {
     int abort_flag;
     // Threshold skip: need[g % NP] == g + 1 when some row of block g kept it, so its PV runs.
     int need[2];
+    // Dynamic tile schedule: the producer takes the next tile index from the launch's counter
+    // and hands it on through this ring (-1: no tile left).  tile_empty counts the MMA warp and
+    // the four softmax warps.
+    uint64_t tile_full[kTileRing3], tile_empty[kTileRing3];
+    int tile_idx[kTileRing3];
     int lst[kListChunk3];
 };
 static_assert(sizeof(Bars3) <= 2048, "barrier region");
@@ -110,6 +116,10 @@ __global__ void __launch_bounds__(kThreads3, 2)
         mbar_init(&bars->o_done[1], 1);
         mbar_init(&bars->drain, 1);
         mbar_init(&bars->tmem_free, 128);
+        for (int t = 0; t < kTileRing3; ++t) {
+            mbar_init(&bars->tile_full[t], 1);
+            mbar_init(&bars->tile_empty[t], 5);
+        }
         bars->abort_flag = 0;
         fence_barrier_init();
         tma_prefetch_desc(&tq);
@@ -128,14 +138,34 @@ __global__ void __launch_bounds__(kThreads3, 2)
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
-        TileIter it;
-        it.init(0, blockIdx.x, gridDim.x, total_tiles);
-        it.next(a);
-        uint32_t ring = 0, qc = 0;
+        uint32_t ring = 0, qc = 0, tn = 0;
         unsigned bad = 0;
         bool ok = true;
-        while (ok && it.active) {
-            const Tile T = it.T;
+        while (ok) {
+            // The next tile of the launch: the first non-empty one at or after the counter.
+            int t = -1;
+            if (lane == 0) {
+                const uint32_t slot = tn % kTileRing3;
+                ok = mbar_wait(&bars->tile_empty[slot], ((tn / kTileRing3) & 1) ^ 1, abort_flag, a.err);
+                if (ok) {
+                    while (true) {
+                        t = atomicAdd(a.tile_counter, 1);
+                        if (t >= total_tiles) {
+                            t = -1;
+                            break;
+                        }
+                        const Tile U = decode_tile(a, t);
+                        if (U.valid && U.n_list > 0) break;
+                    }
+                    bars->tile_idx[slot] = t;
+                    mbar_arrive(&bars->tile_full[slot]);
+                }
+                ++tn;
+            }
+            ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+            t = __shfl_sync(0xFFFFFFFFu, t, 0);
+            if (!ok || t < 0) break;
+            const Tile T = decode_tile(a, t);
             if (lane == 0) {
                 ok = mbar_wait(&bars->q_empty, (qc & 1) ^ 1, abort_flag, a.err);
                 if (ok) {
@@ -155,41 +185,48 @@ __global__ void __launch_bounds__(kThreads3, 2)
                     if (kb + e < T.n_list) bars->lst[e] = list_entry(a, T, kb + e);
                 __syncwarp();
                 if (lane == 0) {
-                    const int kend = min(T.n_list, kb + kListChunk3);
-                    for (int k = kb; ok && k < kend; ++k) {
-                        int j = bars->lst[k - kb];
+                    // K of block j (v = 0) or its V (v = 1) into the next ring stage.
+                    auto issue = [&](int j, int v) -> bool {
                         if (j < 0) {
                             bad |= kDevErrInvalidList;
                             j = 0;
                         }
-                        for (int v = 0; ok && v < 2; ++v) {
-                            const int st = ring % C::NS;
-                            ok = mbar_wait(&bars->kv_empty[st], ((ring / C::NS) & 1) ^ 1, abort_flag, a.err);
-                            if (!ok) break;
-                            uint8_t* dst = smem + C::OFF_RING + st * C::KV_BYTES;
-                            const CUtensorMap* map = v ? &tv : &tk;
-                            uint64_t* fb = &bars->kv_full[st];
-                            mbar_arrive_expect_tx(fb, C::KV_BYTES);
+                        const int st = ring % C::NS;
+                        if (!mbar_wait(&bars->kv_empty[st], ((ring / C::NS) & 1) ^ 1, abort_flag, a.err))
+                            return false;
+                        uint8_t* dst = smem + C::OFF_RING + st * C::KV_BYTES;
+                        const CUtensorMap* map = v ? &tv : &tk;
+                        uint64_t* fb = &bars->kv_full[st];
+                        mbar_arrive_expect_tx(fb, C::KV_BYTES);
 #pragma unroll
-                            for (int p = 0; p < C::QP; ++p) {
-                                if constexpr (PAGED) {
+                        for (int p = 0; p < C::QP; ++p) {
+                            if constexpr (PAGED) {
 #pragma unroll
-                                    for (int pg = 0; pg < BN / 64; ++pg) {
-                                        const int lp = j * (BN / 64) + pg;
-                                        const int phys = physical_page(a, T.b, lp, T.n_tok, bad);
-                                        tma_load_4d(dst + p * BN * 128 + pg * 64 * 128, map, fb, p * C::PW, 0, T.hk, phys);
-                                    }
-                                } else {
-                                    tma_load_4d(dst + p * BN * 128, map, fb, p * C::PW, j * a.block, T.hk, T.b);
+                                for (int pg = 0; pg < BN / 64; ++pg) {
+                                    const int lp = j * (BN / 64) + pg;
+                                    const int phys = physical_page(a, T.b, lp, T.n_tok, bad);
+                                    tma_load_4d(dst + p * BN * 128 + pg * 64 * 128, map, fb, p * C::PW, 0, T.hk, phys);
                                 }
+                            } else {
+                                tma_load_4d(dst + p * BN * 128, map, fb, p * C::PW, j * a.block, T.hk, T.b);
                             }
-                            ++ring;
                         }
+                        ++ring;
+                        return true;
+                    };
+                    // The MMA warp's order: S(0), then S(k+1) ahead of PV(k).  The loads follow it,
+                    // K(0), then K(k+1) before V(k), so a K block is requested one block earlier
+                    // than a V block and the ring is consumed in the order it is filled.
+                    const int kend = min(T.n_list, kb + kListChunk3);
+                    if (kb == 0) ok = issue(bars->lst[0], 0);
+                    for (int k = kb; ok && k < kend; ++k) {
+                        if (k + 1 < T.n_list)
+                            ok = issue(k + 1 < kend ? bars->lst[k + 1 - kb] : list_entry(a, T, k + 1), 0);
+                        if (ok) ok = issue(bars->lst[k - kb], 1);
                     }
                 }
                 ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
             }
-            it.next(a);
         }
         if (lane == 0) {
             if (bad) atomicOr(a.err, bad);
@@ -210,10 +247,20 @@ __global__ void __launch_bounds__(kThreads3, 2)
             uint32_t rbase = 0, qc = 0, pc = 0, sf = 0;
             unsigned long long n_pv_skipped = 0;  // threshold skip: products not issued
             bool ok = true, first_s = true;
-            TileIter it;
-            it.init(0, blockIdx.x, gridDim.x, total_tiles);
-            it.next(a);
-            // S = Q K^T from ring index r (K of a block sits at 2k, its V at 2k + 1).
+            uint32_t tn = 0;
+            Tile T;
+            // The next tile from the producer's ring: 1, or 0 when none is left, -1 on a failed wait.
+            auto next_tile = [&]() -> int {
+                const uint32_t slot = tn % kTileRing3;
+                if (!mbar_wait(&bars->tile_full[slot], (tn / kTileRing3) & 1, abort_flag, a.err)) return -1;
+                const int t = *reinterpret_cast<volatile int*>(&bars->tile_idx[slot]);
+                mbar_arrive(&bars->tile_empty[slot]);
+                ++tn;
+                if (t < 0) return 0;
+                T = decode_tile(a, t);
+                return 1;
+            };
+            // S = Q K^T with K from ring position r.
             auto mma_s = [&](uint32_t r) -> bool {
                 // S is overwritten: the softmax must have read the previous S.
                 if (!first_s) {
@@ -267,22 +314,28 @@ __global__ void __launch_bounds__(kThreads3, 2)
                 tc_commit(&bars->o_done[pb]);
                 return true;
             };
-            while (ok && it.active) {
-                const int n = it.T.n_list;
+            while (ok) {
+                const int nt = next_tile();
+                if (nt <= 0) {
+                    ok = nt == 0;
+                    break;
+                }
+                const int n = T.n_list;
                 ok = mbar_wait(&bars->q_full, qc & 1, abort_flag, a.err);
                 ++qc;
+                // Ring positions of the tile (the producer's order K0, K1, V0, K2, V1, ..., V(n-1)):
+                // K(k) at 2k - 1 for k >= 1, V(k) at 2k + 2 for k < n - 1, V(n - 1) at 2n - 1.
                 ok = ok && mma_s(rbase);
                 if (ok && n == 1) tc_commit(&bars->q_empty);
                 for (int k = 0; ok && k < n; ++k) {
                     // S(k+1) goes ahead of PV(k): it only needs the softmax to have read S(k).
                     if (k + 1 < n) {
-                        ok = mma_s(rbase + 2 * (k + 1));
+                        ok = mma_s(rbase + 2 * k + 1);
                         if (ok && k + 2 == n) tc_commit(&bars->q_empty);  // last S of the tile
                     }
-                    ok = ok && mma_pv(rbase + 2 * k + 1, k > 0);
+                    ok = ok && mma_pv(rbase + (k + 1 < n ? 2 * k + 2 : 2 * n - 1), k > 0);
                 }
                 rbase += 2 * n;
-                it.next(a);
             }
             if (SKIP && a.skip_stats != nullptr) {
                 atomicAdd(a.skip_stats + 2, static_cast<unsigned long long>(pc));
@@ -315,11 +368,20 @@ __global__ void __launch_bounds__(kThreads3, 2)
         const float sl2 = a.scale_log2;
         uint32_t n_vis = 0, n_skipped = 0;  // threshold skip: row-blocks of real rows, and skipped
         bool ok = true;
-        TileIter it;
-        it.init(0, blockIdx.x, gridDim.x, total_tiles);
-        it.next(a);
-        while (ok && it.active) {
-            const Tile T = it.T;
+        uint32_t tn = 0;
+        while (ok) {
+            // The next tile from the producer's ring (every lane waits; lane 0 frees the slot for
+            // the warp once all lanes have read it).
+            const uint32_t tslot = tn % kTileRing3;
+            bool t_ok = mbar_wait(&bars->tile_full[tslot], (tn / kTileRing3) & 1, abort_flag, a.err);
+            t_ok = __all_sync(0xFFFFFFFFu, t_ok);
+            if (!t_ok) break;
+            const int tix = *reinterpret_cast<volatile int*>(&bars->tile_idx[tslot]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->tile_empty[tslot]);
+            ++tn;
+            if (tix < 0) break;
+            const Tile T = decode_tile(a, tix);
             float m_used = -INFINITY, l_run = 0.f;
             float m_true = -INFINITY;  // exact running max (log2 units), for the threshold skip
             // The tile's list, 32 entries per warp-wide load: lane e holds entry 32c + e of the
@@ -531,7 +593,6 @@ __global__ void __launch_bounds__(kThreads3, 2)
                 a.lse[(static_cast<int64_t>(T.b) * a.Hq + T.h) * a.lse_stride + t_row] =
                     (m_used + __log2f(l_run) - kPScale3<FP8>) * 0.69314718055994531f;
             tc_fence_before();
-            it.next(a);
         }
         if (SKIP && a.skip_stats != nullptr) {
             unsigned long long v0 = n_vis, v1 = n_skipped;
@@ -554,6 +615,7 @@ template <bool FP8, int D, int BN, bool PAGED>
 cudaError_t launch_ws3_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const AttnArgs& a,
                          cudaStream_t s) {
     using C = Cfg3<FP8, D, BN>;
+    if (a.tile_counter == nullptr) return cudaErrorInvalidValue;
     auto kern = a.skip_on ? attn_ws3_kernel<FP8, D, BN, PAGED, true> : attn_ws3_kernel<FP8, D, BN, PAGED, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;

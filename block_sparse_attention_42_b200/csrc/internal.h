@@ -88,6 +88,8 @@ struct AttnArgs {
     float* lse;
     int64_t lse_stride;          // tokens per (b, h) row of lse
     unsigned* err;
+    int* tile_counter;           // zeroed before the launch: the next tile index of a dynamic
+                                 // tile schedule (attn_ws3.cu)
 };
 
 // Persistent, two independent pipelined CTAs per SM, one query tile each (attn_ws2.cu).
