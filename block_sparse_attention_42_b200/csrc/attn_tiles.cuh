@@ -4,6 +4,7 @@
 #pragma once
 
 #include "internal.h"
+#include "sm100.cuh"
 
 namespace bsa {
 
@@ -105,4 +106,72 @@ struct TileIter {
     }
 };
 
+// Dynamic tile schedule.  The producer warp takes the next tile index from the launch's
+// counter (a.tile_counter, zeroed before the launch) and hands it to the CTA's other roles
+// through a ring in shared memory; -1 means no tile is left.  Tiles are taken in index order
+// (sequence, KV head, query block from the last, query head), so the heavy tiles go first and
+// each CTA takes the next one when it is free.
+constexpr int kTileRing = 4;
+
+struct TileRing {
+    uint64_t full[kTileRing], empty[kTileRing];
+    int idx[kTileRing];
+};
+
+// One thread, before the CTA's first barrier: `consumers` arrivals free a slot.
+__device__ __forceinline__ void tile_ring_init(TileRing& r, int consumers) {
+    for (int t = 0; t < kTileRing; ++t) {
+        mbar_init(&r.full[t], 1);
+        mbar_init(&r.empty[t], consumers);
+    }
+}
+
+// Producer, one thread: publishes the next non-empty tile at or after the counter (or -1) in
+// slot n % kTileRing.  False when the wait for the slot failed (nothing published).
+__device__ __forceinline__ bool tile_ring_put(TileRing& r, uint32_t n, const AttnArgs& a, int total_tiles, int& t,
+                                              volatile int* abort_flag) {
+    const uint32_t slot = n % kTileRing;
+    if (!mbar_wait(&r.empty[slot], ((n / kTileRing) & 1) ^ 1, abort_flag, a.err)) return false;
+    while (true) {
+        t = atomicAdd(a.tile_counter, 1);
+        if (t >= total_tiles) {
+            t = -1;
+            break;
+        }
+        const Tile U = decode_tile(a, t);
+        if (U.valid && U.n_list > 0) break;
+    }
+    r.idx[slot] = t;
+    mbar_arrive(&r.full[slot]);
+    return true;
+}
+
+// Consumer, one thread: the tile in slot n % kTileRing (frees the slot).  1: a tile, 0: none
+// left, -1: the wait failed.
+__device__ __forceinline__ int tile_ring_get(TileRing& r, uint32_t n, const AttnArgs& a, Tile& T,
+                                             volatile int* abort_flag) {
+    const uint32_t slot = n % kTileRing;
+    if (!mbar_wait(&r.full[slot], (n / kTileRing) & 1, abort_flag, a.err)) return -1;
+    const int t = *reinterpret_cast<volatile int*>(&r.idx[slot]);
+    mbar_arrive(&r.empty[slot]);
+    if (t < 0) return 0;
+    T = decode_tile(a, t);
+    return 1;
+}
+
+// Consumer, a whole warp (every lane waits and reads; lane 0 frees the slot for the warp).
+__device__ __forceinline__ int tile_ring_get_warp(TileRing& r, uint32_t n, const AttnArgs& a, Tile& T,
+                                                  volatile int* abort_flag, int lane) {
+    const uint32_t slot = n % kTileRing;
+    const bool w = __all_sync(0xFFFFFFFFu, mbar_wait(&r.full[slot], (n / kTileRing) & 1, abort_flag, a.err));
+    if (!w) return -1;
+    const int t = *reinterpret_cast<volatile int*>(&r.idx[slot]);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&r.empty[slot]);
+    if (t < 0) return 0;
+    T = decode_tile(a, t);
+    return 1;
+}
+
 }  // namespace bsa
+

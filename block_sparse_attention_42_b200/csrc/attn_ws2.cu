@@ -61,6 +61,7 @@ struct Bars2 {
     uint64_t q_full, q_empty, s_full, p_full, o_done, drain, tmem_free;
     uint32_t tmem_slot;
     int abort_flag;
+    TileRing tiles;  // the dynamic tile schedule; a slot is freed by the MMA and the 4 softmax warps
     int lst[kListChunk2];
 };
 static_assert(sizeof(Bars2) <= 2048, "barrier region");
@@ -88,6 +89,7 @@ __global__ void __launch_bounds__(kThreads2, 2)
         mbar_init(&bars->o_done, 1);
         mbar_init(&bars->drain, 1);
         mbar_init(&bars->tmem_free, 128);
+        tile_ring_init(bars->tiles, 5);
         bars->abort_flag = 0;
         fence_barrier_init();
         tma_prefetch_desc(&tq);
@@ -106,14 +108,17 @@ __global__ void __launch_bounds__(kThreads2, 2)
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
-        TileIter it;
-        it.init(0, blockIdx.x, gridDim.x, total_tiles);
-        it.next(a);
-        uint32_t ring = 0, qc = 0;
+        uint32_t ring = 0, qc = 0, tn = 0;
         unsigned bad = 0;
         bool ok = true;
-        while (ok && it.active) {
-            const Tile T = it.T;
+        while (ok) {
+            // The next tile of the launch, handed on to the MMA and softmax warps.
+            int t = -1;
+            if (lane == 0) ok = tile_ring_put(bars->tiles, tn++, a, total_tiles, t, abort_flag);
+            ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+            t = __shfl_sync(0xFFFFFFFFu, t, 0);
+            if (!ok || t < 0) break;
+            const Tile T = decode_tile(a, t);
             if (lane == 0) {
                 ok = mbar_wait(&bars->q_empty, (qc & 1) ^ 1, abort_flag, a.err);
                 if (ok) {
@@ -167,7 +172,6 @@ __global__ void __launch_bounds__(kThreads2, 2)
                 }
                 ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
             }
-            it.next(a);
         }
         if (lane == 0) {
             if (bad) atomicOr(a.err, bad);
@@ -184,11 +188,9 @@ __global__ void __launch_bounds__(kThreads2, 2)
             const uint32_t idesc_s = make_idesc(kBM2, BN, FP8 ? 0u : 1u, false, false);
             const uint32_t idesc_o = make_idesc(kBM2, D, FP8 ? 0u : 1u, false, true);
             const uint32_t aQ = smem_u32(smem + C::OFF_Q);
-            uint32_t ring = 0, qc = 0, pc = 0;
+            uint32_t ring = 0, qc = 0, pc = 0, tn = 0;
             bool ok = true;
-            TileIter it;
-            it.init(0, blockIdx.x, gridDim.x, total_tiles);
-            it.next(a);
+            Tile T;
             // S = Q K^T from ring stage `ring`
             auto mma_s = [&]() -> bool {
                 const int st = ring % C::NS;
@@ -210,8 +212,13 @@ __global__ void __launch_bounds__(kThreads2, 2)
                 ++ring;
                 return true;
             };
-            while (ok && it.active) {
-                const int n = it.T.n_list;
+            while (ok) {
+                const int nt = tile_ring_get(bars->tiles, tn++, a, T, abort_flag);
+                if (nt <= 0) {
+                    ok = nt == 0;
+                    break;
+                }
+                const int n = T.n_list;
                 ok = mbar_wait(&bars->q_full, qc & 1, abort_flag, a.err);
                 ++qc;
                 ok = ok && mma_s();
@@ -244,7 +251,6 @@ __global__ void __launch_bounds__(kThreads2, 2)
                         if (ok && k + 2 == n) tc_commit(&bars->q_empty);  // last S of the tile
                     }
                 }
-                it.next(a);
             }
             tc_commit(&bars->drain);
             volatile int no_abort = 0;
@@ -265,16 +271,20 @@ __global__ void __launch_bounds__(kThreads2, 2)
         uint32_t scount = 0, ocount = 0;
         const float sl2 = a.scale_log2;
         bool ok = true;
-        TileIter it;
-        it.init(0, blockIdx.x, gridDim.x, total_tiles);
-        it.next(a);
-        while (ok && it.active) {
-            const Tile T = it.T;
+        uint32_t tn = 0;
+        while (ok) {
+            Tile T;
+            if (tile_ring_get_warp(bars->tiles, tn++, a, T, abort_flag, lane) <= 0) break;
             float m_used = -INFINITY, l_run = 0.f;
-            int j_next = list_entry(a, T, 0);
+            // The tile's list, 32 entries per warp-wide load, loaded a chunk ahead of its use.
+            int jl = list_entry_raw(a, T, lane);
+            int jl_next = list_entry_raw(a, T, 32 + lane);
             for (int k = 0; k < T.n_list; ++k) {
-                const int j = j_next;
-                if (k + 1 < T.n_list) j_next = list_entry(a, T, k + 1);
+                if ((k & 31) == 0 && k > 0) {
+                    jl = jl_next;
+                    jl_next = list_entry_raw(a, T, k + 32 + lane);
+                }
+                const int j = list_entry_check(T, __shfl_sync(0xFFFFFFFFu, jl, k & 31));
                 bool w_ok = mbar_wait(&bars->s_full, scount & 1, abort_flag, a.err);
                 ++scount;
                 w_ok = __all_sync(0xFFFFFFFFu, w_ok);
@@ -422,7 +432,6 @@ __global__ void __launch_bounds__(kThreads2, 2)
                 a.lse[(static_cast<int64_t>(T.b) * a.Hq + T.h) * a.lse_stride + t_row] =
                     (m_used + __log2f(l_run) - kPScale2<FP8>) * 0.69314718055994531f;
             tc_fence_before();
-            it.next(a);
         }
         tc_fence_before();
         mbar_arrive(&bars->tmem_free);
@@ -434,6 +443,7 @@ template <bool FP8, int D, int BN, bool PAGED>
 cudaError_t launch_ws2_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const AttnArgs& a,
                          cudaStream_t s) {
     using C = Cfg2<FP8, D, BN>;
+    if (a.tile_counter == nullptr) return cudaErrorInvalidValue;
     auto kern = attn_ws2_kernel<FP8, D, BN, PAGED>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;

@@ -31,7 +31,6 @@ constexpr int kThreads3 = 192;
 constexpr int kSmem3Limit = 115712;  // two CTAs per SM
 constexpr int kMaxStages3 = 6;
 constexpr int kListChunk3 = 128;
-constexpr int kTileRing3 = 4;  // tile indices handed from the producer to the MMA and softmax warps
 
 template <bool FP8, int D, int BN>
 struct Cfg3 {
@@ -80,11 +79,7 @@ struct Bars3 {
     int abort_flag;
     // Threshold skip: need[g % NP] == g + 1 when some row of block g kept it, so its PV runs.
     int need[2];
-    // Dynamic tile schedule: the producer takes the next tile index from the launch's counter
-    // and hands it on through this ring (-1: no tile left).  tile_empty counts the MMA warp and
-    // the four softmax warps.
-    uint64_t tile_full[kTileRing3], tile_empty[kTileRing3];
-    int tile_idx[kTileRing3];
+    TileRing tiles;  // the dynamic tile schedule; a slot is freed by the MMA and the 4 softmax warps
     int lst[kListChunk3];
 };
 static_assert(sizeof(Bars3) <= 2048, "barrier region");
@@ -116,10 +111,7 @@ __global__ void __launch_bounds__(kThreads3, 2)
         mbar_init(&bars->o_done[1], 1);
         mbar_init(&bars->drain, 1);
         mbar_init(&bars->tmem_free, 128);
-        for (int t = 0; t < kTileRing3; ++t) {
-            mbar_init(&bars->tile_full[t], 1);
-            mbar_init(&bars->tile_empty[t], 5);
-        }
+        tile_ring_init(bars->tiles, 5);
         bars->abort_flag = 0;
         fence_barrier_init();
         tma_prefetch_desc(&tq);
@@ -142,26 +134,9 @@ __global__ void __launch_bounds__(kThreads3, 2)
         unsigned bad = 0;
         bool ok = true;
         while (ok) {
-            // The next tile of the launch: the first non-empty one at or after the counter.
+            // The next tile of the launch, handed on to the MMA and softmax warps.
             int t = -1;
-            if (lane == 0) {
-                const uint32_t slot = tn % kTileRing3;
-                ok = mbar_wait(&bars->tile_empty[slot], ((tn / kTileRing3) & 1) ^ 1, abort_flag, a.err);
-                if (ok) {
-                    while (true) {
-                        t = atomicAdd(a.tile_counter, 1);
-                        if (t >= total_tiles) {
-                            t = -1;
-                            break;
-                        }
-                        const Tile U = decode_tile(a, t);
-                        if (U.valid && U.n_list > 0) break;
-                    }
-                    bars->tile_idx[slot] = t;
-                    mbar_arrive(&bars->tile_full[slot]);
-                }
-                ++tn;
-            }
+            if (lane == 0) ok = tile_ring_put(bars->tiles, tn++, a, total_tiles, t, abort_flag);
             ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
             t = __shfl_sync(0xFFFFFFFFu, t, 0);
             if (!ok || t < 0) break;
@@ -249,17 +224,6 @@ __global__ void __launch_bounds__(kThreads3, 2)
             bool ok = true, first_s = true;
             uint32_t tn = 0;
             Tile T;
-            // The next tile from the producer's ring: 1, or 0 when none is left, -1 on a failed wait.
-            auto next_tile = [&]() -> int {
-                const uint32_t slot = tn % kTileRing3;
-                if (!mbar_wait(&bars->tile_full[slot], (tn / kTileRing3) & 1, abort_flag, a.err)) return -1;
-                const int t = *reinterpret_cast<volatile int*>(&bars->tile_idx[slot]);
-                mbar_arrive(&bars->tile_empty[slot]);
-                ++tn;
-                if (t < 0) return 0;
-                T = decode_tile(a, t);
-                return 1;
-            };
             // S = Q K^T with K from ring position r.
             auto mma_s = [&](uint32_t r) -> bool {
                 // S is overwritten: the softmax must have read the previous S.
@@ -315,7 +279,7 @@ __global__ void __launch_bounds__(kThreads3, 2)
                 return true;
             };
             while (ok) {
-                const int nt = next_tile();
+                const int nt = tile_ring_get(bars->tiles, tn++, a, T, abort_flag);
                 if (nt <= 0) {
                     ok = nt == 0;
                     break;
@@ -370,18 +334,8 @@ __global__ void __launch_bounds__(kThreads3, 2)
         bool ok = true;
         uint32_t tn = 0;
         while (ok) {
-            // The next tile from the producer's ring (every lane waits; lane 0 frees the slot for
-            // the warp once all lanes have read it).
-            const uint32_t tslot = tn % kTileRing3;
-            bool t_ok = mbar_wait(&bars->tile_full[tslot], (tn / kTileRing3) & 1, abort_flag, a.err);
-            t_ok = __all_sync(0xFFFFFFFFu, t_ok);
-            if (!t_ok) break;
-            const int tix = *reinterpret_cast<volatile int*>(&bars->tile_idx[tslot]);
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->tile_empty[tslot]);
-            ++tn;
-            if (tix < 0) break;
-            const Tile T = decode_tile(a, tix);
+            Tile T;
+            if (tile_ring_get_warp(bars->tiles, tn++, a, T, abort_flag, lane) <= 0) break;
             float m_used = -INFINITY, l_run = 0.f;
             float m_true = -INFINITY;  // exact running max (log2 units), for the threshold skip
             // The tile's list, 32 entries per warp-wide load: lane e holds entry 32c + e of the
