@@ -885,6 +885,8 @@ bsa_status_t bsa_check_device_error(cudaStream_t stream) {
     if (e != cudaSuccess) return cuda_fail(e, "clear device error word");
     if (v & kDevErrTimeout) return fail(BSA_ERR_TIMEOUT, "a kernel wait ran out of time");
     if (v & kDevErrInvalidList) return fail(BSA_ERR_INVALID_LIST, "a list entry was outside [0, query block]");
+    if (v & kDevErrSmemAlign)
+        return fail(BSA_ERR_CUDA, "an attention kernel found its dynamic shared memory not 1024-byte aligned");
     if (v & kDevErrInvalidPage)
         return fail(BSA_ERR_INVALID_PAGE, "a page-table entry of a token inside its sequence was outside [0, num_pages)");
     return BSA_OK;

@@ -31,6 +31,7 @@ constexpr int kThreads3 = 192;
 constexpr int kSmem3Limit = 115712;  // two CTAs per SM
 constexpr int kMaxStages3 = 6;
 constexpr int kListChunk3 = 128;
+constexpr int kBar3Bytes = 1024;  // barriers, tile ring, list buffer
 
 template <bool FP8, int D, int BN>
 struct Cfg3 {
@@ -41,17 +42,18 @@ struct Cfg3 {
     static constexpr int KV_BYTES = BN * D * EB;
     static constexpr int P_TILE = kBM3 * BN * EB;
     // Two P buffers when four K/V stages still fit beside them: P(k) then waits for PV(k-2),
-    // not PV(k-1).  (With E4M3 at d = 128 the second buffer would cost the fourth stage, which
-    // measured slower on B200.)
-    static constexpr int NP = (kSmem3Limit - 3072 - Q_BYTES - 2 * P_TILE) / KV_BYTES >= 4 ? 2 : 1;
+    // not PV(k-1).  The tiles start at the (1024-byte aligned) base of dynamic shared memory
+    // with the barrier block after them, so E4M3 at d = 128 fits Q, two P buffers and four
+    // stages exactly.
+    static constexpr int NP = (kSmem3Limit - kBar3Bytes - Q_BYTES - 2 * P_TILE) / KV_BYTES >= 4 ? 2 : 1;
     static constexpr int P_BYTES = NP * P_TILE;
-    static constexpr int NS_FIT = (kSmem3Limit - 3072 - Q_BYTES - P_BYTES) / KV_BYTES;
+    static constexpr int NS_FIT = (kSmem3Limit - kBar3Bytes - Q_BYTES - P_BYTES) / KV_BYTES;
     static constexpr int NS = NS_FIT > kMaxStages3 ? kMaxStages3 : NS_FIT;
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_P = Q_BYTES;
     static constexpr int OFF_RING = OFF_P + P_BYTES;
     static constexpr int OFF_BAR = OFF_RING + NS * KV_BYTES;
-    static constexpr int SMEM = OFF_BAR + 2048 + 1024;  // barriers, list buffer + alignment slack
+    static constexpr int SMEM = OFF_BAR + kBar3Bytes;
     static constexpr int KSTEPS_S = D * EB / 32;
     static constexpr int KSTEPS_O = BN * EB / 32;
     static constexpr int ROWS_PER_KSTEP = 32 / EB;
@@ -82,7 +84,7 @@ struct Bars3 {
     TileRing tiles;  // the dynamic tile schedule; a slot is freed by the MMA and the 4 softmax warps
     int lst[kListChunk3];
 };
-static_assert(sizeof(Bars3) <= 2048, "barrier region");
+static_assert(sizeof(Bars3) <= kBar3Bytes, "barrier region");
 
 // SKIP: the threshold-skip instantiation (bsa_prefill_skip); the default one has none of its code.
 template <bool FP8, int D, int BN, bool PAGED, bool SKIP>
@@ -90,8 +92,14 @@ __global__ void __launch_bounds__(kThreads3, 2)
     attn_ws3_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                     const __grid_constant__ CUtensorMap tv, const AttnArgs a, int total_tiles) {
     using C = Cfg3<FP8, D, BN>;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // The 128-byte-swizzled tiles need 1024-byte alignment and there is no slack to align up:
+    // a base that is not aligned is reported (no thread has touched anything yet).
+    if (smem_u32(smem_raw) & 1023u) {
+        if (threadIdx.x == 0) atomicOr(a.err, kDevErrSmemAlign);
+        return;
+    }
+    uint8_t* smem = smem_raw;
     Bars3* bars = reinterpret_cast<Bars3*>(smem + C::OFF_BAR);
     volatile int* abort_flag = &bars->abort_flag;
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;

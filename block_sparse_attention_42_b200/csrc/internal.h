@@ -12,6 +12,7 @@ namespace bsa {
 constexpr unsigned kDevErrInvalidList = 1u;
 constexpr unsigned kDevErrTimeout = 2u;
 constexpr unsigned kDevErrInvalidPage = 4u;
+constexpr unsigned kDevErrSmemAlign = 8u;  // dynamic shared memory not 1024-byte aligned (nothing ran)
 
 constexpr int kMaxBatch = 256;     // sequences per call
 constexpr int kMaxBlocks = 2048;   // query blocks per sequence
