@@ -375,13 +375,12 @@ __global__ void __launch_bounds__(kThreads3, 2)
 #pragma unroll
                 for (int q = 0; q < 8; ++q) m8[q] = -INFINITY;
                 auto mask_max = [&](int base) {
-                    if (diag) {
+                    if (diag || j < 0) {
+                        // keys past lim are masked: the causal part of the diagonal block, or all
+                        const int lim = j < 0 ? -1 : row - base;
 #pragma unroll
                         for (int e = 0; e < 64; ++e)
-                            if (base + e > row) rr[base + e] = __float_as_uint(-INFINITY);
-                    } else if (j < 0) {
-#pragma unroll
-                        for (int e = 0; e < 64; ++e) rr[base + e] = __float_as_uint(-INFINITY);
+                            if (e > lim) rr[base + e] = __float_as_uint(-INFINITY);
                     }
 #pragma unroll
                     for (int e = 0; e < 64; e += 2)
