@@ -575,7 +575,7 @@ def run_ours(args, rank, world, device):
         bsa.bsa_check_device_error(device)
         same = bool(torch.equal(f_rp, row_ptr) and torch.equal(f_ci, col_idx))
         res["fused_select"] = {"what": "stem_score_select: pool, budget, then per chunk of KV-head groups the score "
-                                       "GEMM into an L2-sized scratch and the top-k from it; no score matrix",
+                                       "GEMM into a scratch of at most 128 MiB and the top-k from it; no score matrix",
                                "ms": f_ms, "unfused_select_ms": res["select_ms"], "lists_equal_unfused": same,
                                "workspace_bytes": f_ws.numel(),
                                "unfused_bytes": scores.numel() * 4 + ws.numel()}

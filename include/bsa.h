@@ -128,7 +128,7 @@ bsa_status_t stem_select(const float* scores, int32_t B, int32_t Hq, const int32
  * exactly what stem_score followed by stem_select computes (the same lists, bit for bit: the
  * same per-tile score products and the same per-row selection), for B sequences of N tokens
  * (nb = ceil(N / block) blocks each), without a [B, Hq, nb, nb] score buffer.  The scores of one
- * chunk of KV-head groups of one sequence exist at a time, in `ws` (at most 64 MiB of it, or one
+ * chunk of KV-head groups of one sequence exist at a time, in `ws` (at most 128 MiB of it, or one
  * group when a group alone is larger), and are consumed by the top-k before the next chunk is
  * scored.  Outputs: row_ptr [B, nb + 1] and col_idx [B, Hq, max_k] as stem_select writes them;
  * max_k >= bsa_tpd_budget(nb, density, tpd_decay, NULL).  ws: at least
