@@ -483,11 +483,18 @@ __global__ void __launch_bounds__(kThreads3, 2)
                     }
                 }
                 fence_proxy_async_smem();
+                float s0, s1, s2, s3, s4, s5, s6, s7;
+                unpack_f32x2(sum4[0], s0, s1);
+                unpack_f32x2(sum4[1], s2, s3);
+                unpack_f32x2(sum4[2], s4, s5);
+                unpack_f32x2(sum4[3], s6, s7);
+                const float sum = ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
                 float alpha = 1.f;
                 if (k > 0 && __any_sync(0xFFFFFFFFu, moved)) {
-                    // O *= alpha once PV(k-1) has finished accumulating into it, 64 TMEM columns at
-                    // a time (P is in shared memory, rr is free).  (At k = 0 there is no O yet and
-                    // l_run is 0, so the factor is not needed.)
+                    // O *= alpha once PV(k-1) has finished accumulating into it.  P is in shared
+                    // memory, so rr is free: both 64-column halves of the O row are read at once
+                    // (the partial sums were reduced above to leave the registers for them).  (At
+                    // k = 0 there is no O yet and l_run is 0, so the factor is not needed.)
                     if (moved) alpha = fast_exp2(m_used - m_new);
                     if (C::NP > 1) {
                         if (!wait_pv(g - 1)) {
@@ -497,10 +504,7 @@ __global__ void __launch_bounds__(kThreads3, 2)
                         tc_fence_after();
                     }
                     const uint64_t a2 = pack_f32x2(alpha, alpha);
-#pragma unroll 1
-                    for (int ch = 0; ch < D / 64; ++ch) {
-                        uint32_t ro[64];
-                        tmem_ld64(tO + ch * 64, ro);
+                    auto scale64 = [&](uint32_t(&ro)[64]) {
 #pragma unroll
                         for (int e = 0; e < 64; e += 2) {
                             float v0, v1;
@@ -508,15 +512,28 @@ __global__ void __launch_bounds__(kThreads3, 2)
                             ro[e] = __float_as_uint(v0);
                             ro[e + 1] = __float_as_uint(v1);
                         }
-                        tmem_st64(tO + ch * 64, ro);
+                    };
+                    if constexpr (D == 128 && BN == 128) {
+                        uint32_t(&ra)[64] = *reinterpret_cast<uint32_t(*)[64]>(rr);
+                        uint32_t(&rb)[64] = *reinterpret_cast<uint32_t(*)[64]>(rr + 64);
+                        tmem_ld64_nowait(tO, ra);
+                        tmem_ld64_nowait(tO + 64, rb);
+                        tmem_ld_wait64(rb);
+                        tmem_ld_wait64(ra);
+                        scale64(ra);
+                        scale64(rb);
+                        tmem_st64(tO, ra);
+                        tmem_st64(tO + 64, rb);
+                    } else {
+#pragma unroll 1
+                        for (int ch = 0; ch < D / 64; ++ch) {
+                            uint32_t ro[64];
+                            tmem_ld64(tO + ch * 64, ro);
+                            scale64(ro);
+                            tmem_st64(tO + ch * 64, ro);
+                        }
                     }
                 }
-                float s0, s1, s2, s3, s4, s5, s6, s7;
-                unpack_f32x2(sum4[0], s0, s1);
-                unpack_f32x2(sum4[1], s2, s3);
-                unpack_f32x2(sum4[2], s4, s5);
-                unpack_f32x2(sum4[3], s6, s7);
-                const float sum = ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
                 l_run = l_run * alpha + sum;
                 m_used = m_new;
                 tmem_st_wait();
