@@ -392,10 +392,16 @@ __global__ void __launch_bounds__(kThreadsG, 1)
         const Tile T = it.T;
         const int h = T.h + slot;
         float m_used = -INFINITY, l_run = 0.f;
-        int j_next = list_entry(a, T, 0);
+        // The unit's list, 32 entries per warp-wide load (lane e: entry 32c + e), a chunk ahead of
+        // its use; block k's entry is a shuffle.
+        int jl = list_entry_raw(a, T, lane);
+        int jl_next = list_entry_raw(a, T, 32 + lane);
         for (int k = 0; k < T.n_list; ++k) {
-            const int j = j_next;
-            if (k + 1 < T.n_list) j_next = list_entry(a, T, k + 1);
+            if ((k & 31) == 0 && k > 0) {
+                jl = jl_next;
+                jl_next = list_entry_raw(a, T, k + 32 + lane);
+            }
+            const int j = list_entry_check(T, __shfl_sync(0xFFFFFFFFu, jl, k & 31));
             bool w_ok = mbar_wait(&B.s_full, scount & 1, abort_flag, a.err);
             ++scount;
             w_ok = __all_sync(0xFFFFFFFFu, w_ok);
@@ -414,13 +420,12 @@ __global__ void __launch_bounds__(kThreadsG, 1)
 #pragma unroll
             for (int q = 0; q < 8; ++q) m8[q] = -INFINITY;
             auto mask_max = [&](int base) {
-                if (diag) {
+                if (diag || j < 0) {
+                    // keys past lim are masked: the causal part of the diagonal block, or all
+                    const int lim = j < 0 ? -1 : row - base;
 #pragma unroll
                     for (int e = 0; e < 64; ++e)
-                        if (base + e > row) rr[base + e] = __float_as_uint(-INFINITY);
-                } else if (j < 0) {
-#pragma unroll
-                    for (int e = 0; e < 64; ++e) rr[base + e] = __float_as_uint(-INFINITY);
+                        if (e > lim) rr[base + e] = __float_as_uint(-INFINITY);
                 }
 #pragma unroll
                 for (int e = 0; e < 64; e += 2)
@@ -438,7 +443,7 @@ __global__ void __launch_bounds__(kThreadsG, 1)
             const float m_blk = mx * sl2;
             float m_new = m_used;
             if (m_blk > m_used + kRescaleG) m_new = m_blk;
-            const float alpha = (m_new == m_used) ? 1.f : fast_exp2(m_used - m_new);
+            const bool moved = m_new != m_used;
             const float mref = (m_new == -INFINITY) ? 0.f : m_new - kPScaleG;
             // Wait for this slot's turn (bounded: past the limit it goes on without it).
             {
@@ -487,42 +492,49 @@ __global__ void __launch_bounds__(kThreadsG, 1)
                     make_uint4(w4[0], w4[1], w4[2], w4[3]);
             }
             fence_proxy_async_smem();
-            bool rescaled = false;
-            if (k > 0 && __any_sync(0xFFFFFFFFu, alpha != 1.f)) {
-                // O *= alpha once PV(g - 1) has finished accumulating into it, 64 TMEM columns at
-                // a time.
-                if (!wait_pv(g - 1)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                const uint64_t a2 = pack_f32x2(alpha, alpha);
-#pragma unroll 1
-                for (int ch = 0; ch < D / 64; ++ch) {
-                    uint32_t ro[64];
-                    tmem_ld64(tO + ch * 64, ro);
-#pragma unroll
-                    for (int e = 0; e < 64; e += 2) {
-                        float v0, v1;
-                        unpack_f32x2(mul_f32x2(pack_f32x2(__uint_as_float(ro[e]), __uint_as_float(ro[e + 1])), a2),
-                                     v0, v1);
-                        ro[e] = __float_as_uint(v0);
-                        ro[e + 1] = __float_as_uint(v1);
-                    }
-                    tmem_st64(tO + ch * 64, ro);
-                }
-                rescaled = true;
-            }
-            if (rescaled) tmem_st_wait();
-            tc_fence_before();
-            mbar_arrive(&B.p_full[g % C::NP]);
-            ++g;
             float s0, s1, s2, s3, s4, s5, s6, s7;
             unpack_f32x2(sum4[0], s0, s1);
             unpack_f32x2(sum4[1], s2, s3);
             unpack_f32x2(sum4[2], s4, s5);
             unpack_f32x2(sum4[3], s6, s7);
             const float sum = ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
+            bool rescaled = false;
+            float alpha = 1.f;
+            if (k > 0 && __any_sync(0xFFFFFFFFu, moved)) {
+                // O *= alpha once PV(g - 1) has finished accumulating into it; both 64-column
+                // halves of the O row at once (P is in shared memory, rr is free).  (At k = 0
+                // there is no O yet and l_run is 0, so the factor is not needed.)
+                if (moved) alpha = fast_exp2(m_used - m_new);
+                if (!wait_pv(g - 1)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint64_t a2 = pack_f32x2(alpha, alpha);
+                uint32_t(&ra)[64] = *reinterpret_cast<uint32_t(*)[64]>(rr);
+                uint32_t(&rb)[64] = *reinterpret_cast<uint32_t(*)[64]>(rr + 64);
+                tmem_ld64_nowait(tO, ra);
+                tmem_ld64_nowait(tO + 64, rb);
+                tmem_ld_wait64(rb);
+                tmem_ld_wait64(ra);
+#pragma unroll
+                for (int e = 0; e < 64; e += 2) {
+                    float v0, v1;
+                    unpack_f32x2(mul_f32x2(pack_f32x2(__uint_as_float(ra[e]), __uint_as_float(ra[e + 1])), a2), v0, v1);
+                    ra[e] = __float_as_uint(v0);
+                    ra[e + 1] = __float_as_uint(v1);
+                    unpack_f32x2(mul_f32x2(pack_f32x2(__uint_as_float(rb[e]), __uint_as_float(rb[e + 1])), a2), v0, v1);
+                    rb[e] = __float_as_uint(v0);
+                    rb[e + 1] = __float_as_uint(v1);
+                }
+                tmem_st64(tO, ra);
+                tmem_st64(tO + 64, rb);
+                rescaled = true;
+            }
+            if (rescaled) tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(&B.p_full[g % C::NP]);
+            ++g;
             l_run = l_run * alpha + sum;
             m_used = m_new;
         }
