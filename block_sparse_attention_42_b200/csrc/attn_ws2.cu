@@ -294,98 +294,67 @@ __global__ void __launch_bounds__(kThreads2, 2)
                 }
                 tc_fence_after();
                 const bool diag = (j == T.i);
-                // Pass 1: row max, 64 TMEM columns per load, eight independent max chains.
-                float mx = -INFINITY;
-                if (j >= 0) {
-                    float m8[8];
+                // The S row in registers, one TMEM read.  Masked scores become -inf before the
+                // max: the causal part of the diagonal block, all of a skipped block.
+                uint32_t rr[BN];
+                float m8[8];
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) m8[q] = -INFINITY;
+                for (int q = 0; q < 8; ++q) m8[q] = -INFINITY;
+                auto mask_max = [&](int base) {
+                    if (diag || j < 0) {
+                        const int lim = j < 0 ? -1 : row - base;  // keys past lim are masked
 #pragma unroll
-                    for (int hf = 0; hf < BN / 64; ++hf) {
-                        uint32_t rr[64];
-                        tmem_ld64(tS + hf * 64, rr);
-                        if (!diag) {
-#pragma unroll
-                            for (int e = 0; e < 64; e += 2)
-                                m8[(e / 2) % 8] = max3f(m8[(e / 2) % 8], __uint_as_float(rr[e]), __uint_as_float(rr[e + 1]));
-                        } else {
-#pragma unroll
-                            for (int e = 0; e < 64; ++e)
-                                if (hf * 64 + e <= row) m8[e % 8] = fmaxf(m8[e % 8], __uint_as_float(rr[e]));
-                        }
+                        for (int e = 0; e < 64; ++e)
+                            if (e > lim) rr[base + e] = __float_as_uint(-INFINITY);
                     }
-                    mx = max3f(max3f(m8[0], m8[1], m8[2]), max3f(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
+#pragma unroll
+                    for (int e = 0; e < 64; e += 2)
+                        m8[(e / 2) % 8] = max3f(m8[(e / 2) % 8], __uint_as_float(rr[base + e]), __uint_as_float(rr[base + e + 1]));
+                };
+                if constexpr (BN == 128) {
+                    // (one 128-column read: overlapping the halves spills at this register budget)
+                    tmem_ld128(tS, rr);
+                    mask_max(0);
+                    mask_max(64);
+                } else {
+                    tmem_ld64(tS, *reinterpret_cast<uint32_t(*)[64]>(rr));
+                    mask_max(0);
                 }
+                const float mx = max3f(max3f(m8[0], m8[1], m8[2]), max3f(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
                 const float m_blk = mx * sl2;
                 float m_new = m_used;
                 if (m_blk > m_used + kRescale2<FP8>) m_new = m_blk;
-                const float alpha = (m_new == m_used) ? 1.f : fast_exp2(m_used - m_new);
+                const bool moved = m_new != m_used;
                 const float mref = (m_new == -INFINITY) ? 0.f : m_new - kPScale2<FP8>;
-                if (k > 0) {
-                    w_ok = mbar_wait(&bars->o_done, ocount & 1, abort_flag, a.err);
-                    ++ocount;
-                    w_ok = __all_sync(0xFFFFFFFFu, w_ok);
-                    if (!w_ok) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    if (__any_sync(0xFFFFFFFFu, alpha != 1.f)) {
-#pragma unroll 1
-                        for (int ch = 0; ch < D / 32; ++ch) {
-                            uint32_t ro[32];
-                            tmem_ld32(tO + ch * 32, ro);
-#pragma unroll
-                            for (int e = 0; e < 32; ++e) ro[e] = __float_as_uint(__uint_as_float(ro[e]) * alpha);
-                            tmem_st32(tO + ch * 32, ro);
-                        }
-                    }
-                }
-                // Pass 2: P = exp2(S * sl2 - mref), 64 columns at a time; P is packed (BF16 pairs
-                // or E4M3 quads) over the S columns already read, as the TMEM A operand of PV.
+                // P = exp2(S * sl2 - mref) in place, four packed partial sums.
                 const uint64_t sl2x2 = pack_f32x2(sl2, sl2);
                 const uint64_t negm = pack_f32x2(-mref, -mref);
                 uint64_t sum4[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-                for (int hf = 0; hf < BN / 64; ++hf) {
-                    uint32_t rr[64];
-                    tmem_ld64(tS + hf * 64, rr);
-                    // Masked scores become -inf outside the exponential loop.
-                    if (diag) {
+                for (int e = 0; e < BN; e += 2) {
+                    const uint64_t x = fma_f32x2(pack_f32x2(__uint_as_float(rr[e]), __uint_as_float(rr[e + 1])), sl2x2, negm);
+                    float x0, x1;
+                    unpack_f32x2(x, x0, x1);
+                    const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+                    sum4[(e / 2) % 4] = add_f32x2(sum4[(e / 2) % 4], pack_f32x2(p0, p1));
+                    rr[e] = __float_as_uint(p0);
+                    rr[e + 1] = __float_as_uint(p1);
+                }
+                // P packed (BF16 pairs or E4M3 quads) over the S columns, as the TMEM A operand
+                // of PV (S(k) was computed after PV(k-1) had read P(k-1) from them).
+                // (8 TMEM columns per store, so few registers beyond the P row are live)
 #pragma unroll
-                        for (int e = 0; e < 64; ++e)
-                            if (hf * 64 + e > row) rr[e] = __float_as_uint(-INFINITY);
-                    } else if (j < 0) {
+                for (int c = 0; c < BN / (FP8 ? 32 : 16); ++c) {
+                    uint32_t pk[8];
 #pragma unroll
-                        for (int e = 0; e < 64; ++e) rr[e] = __float_as_uint(-INFINITY);
+                    for (int q = 0; q < 8; ++q) {
+                        if constexpr (FP8)
+                            pk[q] = pack_e4m3x4(__uint_as_float(rr[c * 32 + 4 * q]), __uint_as_float(rr[c * 32 + 4 * q + 1]),
+                                                __uint_as_float(rr[c * 32 + 4 * q + 2]), __uint_as_float(rr[c * 32 + 4 * q + 3]));
+                        else
+                            pk[q] = pack_bf16x2(__uint_as_float(rr[c * 16 + 2 * q]), __uint_as_float(rr[c * 16 + 2 * q + 1]));
                     }
-#pragma unroll
-                    for (int e = 0; e < 64; e += 2) {
-                        const uint64_t x = fma_f32x2(pack_f32x2(__uint_as_float(rr[e]), __uint_as_float(rr[e + 1])),
-                                                     sl2x2, negm);
-                        float x0, x1;
-                        unpack_f32x2(x, x0, x1);
-                        const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
-                        sum4[(e / 2) % 4] = add_f32x2(sum4[(e / 2) % 4], pack_f32x2(p0, p1));
-                        rr[e] = __float_as_uint(p0);
-                        rr[e + 1] = __float_as_uint(p1);
-                    }
-                    if constexpr (FP8) {
-                        uint32_t pk[16];
-#pragma unroll
-                        for (int q = 0; q < 16; ++q)
-                            pk[q] = pack_e4m3x2(__uint_as_float(rr[4 * q]), __uint_as_float(rr[4 * q + 1])) |
-                                    (static_cast<uint32_t>(pack_e4m3x2(__uint_as_float(rr[4 * q + 2]),
-                                                                       __uint_as_float(rr[4 * q + 3])))
-                                     << 16);
-                        tmem_st16(tS + hf * 16, pk);
-                    } else {
-                        uint32_t pk[32];
-#pragma unroll
-                        for (int q = 0; q < 32; ++q)
-                            pk[q] = pack_bf16x2(__uint_as_float(rr[2 * q]), __uint_as_float(rr[2 * q + 1]));
-                        tmem_st32(tS + hf * 32, pk);
-                    }
+                    tmem_st8(tS + c * 8, pk);
                 }
                 float s0, s1, s2, s3, s4, s5, s6, s7;
                 unpack_f32x2(sum4[0], s0, s1);
@@ -393,6 +362,53 @@ __global__ void __launch_bounds__(kThreads2, 2)
                 unpack_f32x2(sum4[2], s4, s5);
                 unpack_f32x2(sum4[3], s6, s7);
                 const float sum = ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
+                float alpha = 1.f;
+                if (k > 0) {
+                    // PV(k-1) has finished accumulating into O (the commit of S(k) already implies
+                    // it: the two were issued in that order by one thread).
+                    w_ok = mbar_wait(&bars->o_done, ocount & 1, abort_flag, a.err);
+                    ++ocount;
+                    if (!__all_sync(0xFFFFFFFFu, w_ok)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    if (__any_sync(0xFFFFFFFFu, moved)) {
+                        // O *= alpha, the O row read 64 columns at a time, both halves at once
+                        // where D = 128 and rr (128 registers, P already in TMEM) holds them.
+                        if (moved) alpha = fast_exp2(m_used - m_new);
+                        const uint64_t a2 = pack_f32x2(alpha, alpha);
+                        auto scale64 = [&](uint32_t(&ro)[64]) {
+#pragma unroll
+                            for (int e = 0; e < 64; e += 2) {
+                                float v0, v1;
+                                unpack_f32x2(mul_f32x2(pack_f32x2(__uint_as_float(ro[e]), __uint_as_float(ro[e + 1])), a2), v0, v1);
+                                ro[e] = __float_as_uint(v0);
+                                ro[e + 1] = __float_as_uint(v1);
+                            }
+                        };
+                        if constexpr (D == 128 && BN == 128) {
+                            uint32_t(&ra)[64] = *reinterpret_cast<uint32_t(*)[64]>(rr);
+                            uint32_t(&rb)[64] = *reinterpret_cast<uint32_t(*)[64]>(rr + 64);
+                            tmem_ld64_nowait(tO, ra);
+                            tmem_ld64_nowait(tO + 64, rb);
+                            tmem_ld_wait64(rb);
+                            tmem_ld_wait64(ra);
+                            scale64(ra);
+                            scale64(rb);
+                            tmem_st64(tO, ra);
+                            tmem_st64(tO + 64, rb);
+                        } else {
+#pragma unroll 1
+                            for (int ch = 0; ch < D / 64; ++ch) {
+                                uint32_t ro[64];
+                                tmem_ld64(tO + ch * 64, ro);
+                                scale64(ro);
+                                tmem_st64(tO + ch * 64, ro);
+                            }
+                        }
+                    }
+                }
                 l_run = l_run * alpha + sum;
                 m_used = m_new;
                 tmem_st_wait();
