@@ -158,7 +158,7 @@ def whole_job_tflops(eff_flop_per_rank: float, world: int, ms_per_step: float) -
 # linear in B x N.  Keyed by attention kernel and (dtype, Hq, Hkv, d) of the capture; any
 # other kernel or shape reports null.
 TRAFFIC_PER_TOKEN = {
-    ("ws3", "fp8", 64, 8, 128): (358.977536e6 + 484.839168e6) / 32768,
+    ("ws3", "fp8", 64, 8, 128): (358.912512e6 + 485.153280e6) / 32768,
 }
 ATTN_DEFAULT = "ws3"  # the kernel bsa_prefill runs when BSA_ATTN_VARIANT is unset
 

@@ -42,7 +42,7 @@ def test_throughput_and_traffic_helpers(monkeypatch):
     # DRAM traffic of the default kernel is linear in tokens; other kernels / shapes report null
     monkeypatch.delenv("BSA_ATTN_VARIANT", raising=False)
     t1 = bench.attn_traffic(True, 1, 32768, 64, 8, 128)
-    assert t1 == pytest.approx(358.977536e6 + 484.839168e6)
+    assert t1 == pytest.approx(358.912512e6 + 485.153280e6)
     assert bench.attn_traffic(True, 1, 131072, 64, 8, 128) == pytest.approx(4 * t1)
     assert bench.attn_traffic(True, 2, 32768, 64, 8, 128) == pytest.approx(2 * t1)
     assert bench.attn_traffic(False, 1, 32768, 64, 8, 128) is None
