@@ -36,7 +36,8 @@
  *   - Calls are asynchronous on `stream`.  Argument errors are returned synchronously, with
  *     nothing launched, and the message is available from bsa_last_error().  A failed launch
  *     returns BSA_ERR_CUDA.  Errors found by kernels while running (an out-of-range list
- *     entry, an out-of-range page-table entry, an internal wait that ran out of time) are
+ *     entry, an out-of-range page-table entry, an internal wait that ran out of time, a
+ *     dynamic shared-memory base without the 1024-byte alignment the attention tiles need) are
  *     recorded in a per-device error word that bsa_check_device_error() reads.
  *   - Tensors are described by bsa_tensor_t: element strides of batch, token and head; the
  *     feature (head_dim) dimension is contiguous; the base pointer and every stride must be
@@ -305,8 +306,9 @@ bsa_status_t bsa_selftest_wait_timeout(uint64_t limit_ns, cudaStream_t stream);
 const char* bsa_last_error(void);
 
 /* Synchronises `stream`, then reads and clears the current device's error word: returns
- * BSA_ERR_TIMEOUT, BSA_ERR_INVALID_LIST or BSA_ERR_INVALID_PAGE if a kernel recorded one (in
- * that order of precedence), else BSA_OK. */
+ * BSA_ERR_TIMEOUT, BSA_ERR_INVALID_LIST, BSA_ERR_CUDA (an attention kernel found its dynamic
+ * shared memory not 1024-byte aligned and did nothing) or BSA_ERR_INVALID_PAGE if a kernel
+ * recorded one (in that order of precedence), else BSA_OK. */
 bsa_status_t bsa_check_device_error(cudaStream_t stream);
 
 #ifdef __cplusplus
