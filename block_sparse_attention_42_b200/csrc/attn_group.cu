@@ -12,8 +12,10 @@
 // pair of query heads of the group).  The pair's two heads are the two slots.  Registers are
 // split by warpgroup with setmaxnreg: the control warpgroup (warps 0-3) drops to 56 per thread,
 // the two softmax warpgroups rise to 224.
-//   warp 0      TMA producer: both slots' Q tiles of each unit (one transaction), then K_j and
-//               V_j of every kept block into one ring of stages shared by the slots
+//   warp 0      TMA producer: takes the next unit from the launch's counter (handing it to the
+//               other roles through a ring in shared memory), loads both slots' Q tiles of the
+//               unit (one transaction), then K_j and V_j of every kept block into one ring of
+//               stages shared by the slots, in the order the MMA warps consume them
 //   warps 1, 3  MMA issuers of slot 0 and slot 1 (warp 1 owns tensor memory): S(k+1) = Q K^T as
 //               soon as the slot's softmax has read S(k), O += P(k) V once P(k) is in shared
 //               memory.  A ring stage is free once both slots' products have read it.
@@ -25,7 +27,8 @@
 // exponential phases would run at the same time: the MUFU (16 ex2 per clock per SM) would be
 // shared while both exponentiate and idle while both do the rest of a block.  A token makes the
 // slots take turns at the exponentials, so one slot's exponentials overlap the other's loads,
-// max, P stores and rescale (measured at fp8-128k: 52.3 ms against 56.7 ms without it).
+// max, P stores and rescale (measured at fp8-128k, before later changes: 52.3 ms against 56.7 ms
+// without it).
 // Tensor memory (512 columns): S slot 0 | S slot 1 | O slot 0 | O slot 1.
 #include <cuda_bf16.h>
 
@@ -96,6 +99,7 @@ struct BarsG {
     uint64_t turn[kSlotsG];
     uint32_t tmem_slot;
     int abort_flag;
+    TileRing units;        // the dynamic unit schedule; freed by both MMA warps and 8 softmax warps
     int lst[kListChunkG];  // list entries staged by the producer warp
 };
 static_assert(sizeof(BarsG) <= 2048, "barrier region");
@@ -110,30 +114,10 @@ __device__ __forceinline__ int unit_to_tile(const AttnArgs& a, int u) {
     return b * a.Hkv * a.nb_max * G + y * G + 2 * p;
 }
 
-// The static walk over work units of one CTA: units base, base + stride, ... that are not empty.
-struct UnitIter {
-    int round, base, stride, total;
-    bool active;
-    Tile T;  // of the pair's first head (T.h); the second head is T.h + 1
-    __device__ __forceinline__ void init(int base_, int stride_, int total_) {
-        base = base_;
-        stride = stride_;
-        total = total_;
-        round = 0;
-        active = true;
-    }
-    __device__ __forceinline__ void next(const AttnArgs& a) {
-        while (true) {
-            const int u = base + round * stride;
-            ++round;
-            if (u >= total) {
-                active = false;
-                return;
-            }
-            T = decode_tile(a, unit_to_tile(a, u));
-            if (T.valid && T.n_list > 0) return;
-        }
-    }
+// The launch's counter runs over units; the ring carries the tile of the pair's first head.
+struct UnitToTile {
+    const AttnArgs* a;
+    __device__ __forceinline__ int operator()(int u) const { return unit_to_tile(*a, u); }
 };
 
 template <bool PAGED>
@@ -169,6 +153,7 @@ __global__ void __launch_bounds__(kThreadsG, 1)
         mbar_init(&bars->tmem_free, 256);
         mbar_init(&bars->turn[0], 128);
         mbar_init(&bars->turn[1], 128);
+        tile_ring_init(bars->units, 2 + 8);
         bars->abort_flag = 0;
         fence_barrier_init();
         tma_prefetch_desc(&tq);
@@ -191,14 +176,17 @@ __global__ void __launch_bounds__(kThreadsG, 1)
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kRegsCtrlG));
         if (warp == 0) {
             // ------------------------------------------------------------ TMA producer
-            UnitIter it;
-            it.init(blockIdx.x, gridDim.x, total_units);
-            it.next(a);
-            uint32_t ring = 0, qc = 0;
+            uint32_t ring = 0, qc = 0, tn = 0;
             unsigned bad = 0;
             bool ok = true;
-            while (ok && it.active) {
-                const Tile T = it.T;
+            while (ok) {
+                // The next unit of the launch, handed on to the MMA and softmax warps.
+                int t = -1;
+                if (lane == 0) ok = tile_ring_put(bars->units, tn++, a, total_units, t, abort_flag, UnitToTile{&a});
+                ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+                t = __shfl_sync(0xFFFFFFFFu, t, 0);
+                if (!ok || t < 0) break;
+                const Tile T = decode_tile(a, t);  // of the pair's first head; the second is T.h + 1
                 if (lane == 0) {
                     ok = mbar_wait(&bars->q_empty, (qc & 1) ^ 1, abort_flag, a.err);
                     if (ok) {
@@ -219,42 +207,49 @@ __global__ void __launch_bounds__(kThreadsG, 1)
                         if (kb + e < T.n_list) bars->lst[e] = list_entry(a, T, kb + e);
                     __syncwarp();
                     if (lane == 0) {
-                        const int kend = min(T.n_list, kb + kListChunkG);
-                        for (int k = kb; ok && k < kend; ++k) {
-                            int j = bars->lst[k - kb];
+                        // K of block j (v = 0) or its V (v = 1) into the next ring stage.
+                        auto issue = [&](int j, int v) -> bool {
                             if (j < 0) {
                                 bad |= kDevErrInvalidList;
                                 j = 0;
                             }
-                            for (int v = 0; ok && v < 2; ++v) {
-                                const int st = ring % C::NS;
-                                ok = mbar_wait(&bars->kv_empty[st], ((ring / C::NS) & 1) ^ 1, abort_flag, a.err);
-                                if (!ok) break;
-                                uint8_t* dst = smem + C::OFF_RING + st * C::KV_BYTES;
-                                const CUtensorMap* map = v ? &tv : &tk;
-                                uint64_t* fb = &bars->kv_full[st];
-                                mbar_arrive_expect_tx(fb, C::KV_BYTES);
+                            const int st = ring % C::NS;
+                            if (!mbar_wait(&bars->kv_empty[st], ((ring / C::NS) & 1) ^ 1, abort_flag, a.err))
+                                return false;
+                            uint8_t* dst = smem + C::OFF_RING + st * C::KV_BYTES;
+                            const CUtensorMap* map = v ? &tv : &tk;
+                            uint64_t* fb = &bars->kv_full[st];
+                            mbar_arrive_expect_tx(fb, C::KV_BYTES);
 #pragma unroll
-                                for (int p = 0; p < C::QP; ++p) {
-                                    if constexpr (PAGED) {
+                            for (int p = 0; p < C::QP; ++p) {
+                                if constexpr (PAGED) {
 #pragma unroll
-                                        for (int pg = 0; pg < BN / 64; ++pg) {
-                                            const int lp = j * (BN / 64) + pg;
-                                            const int phys = physical_page(a, T.b, lp, T.n_tok, bad);
-                                            tma_load_4d(dst + p * BN * 128 + pg * 64 * 128, map, fb, p * C::PW, 0,
-                                                        T.hk, phys);
-                                        }
-                                    } else {
-                                        tma_load_4d(dst + p * BN * 128, map, fb, p * C::PW, j * a.block, T.hk, T.b);
+                                    for (int pg = 0; pg < BN / 64; ++pg) {
+                                        const int lp = j * (BN / 64) + pg;
+                                        const int phys = physical_page(a, T.b, lp, T.n_tok, bad);
+                                        tma_load_4d(dst + p * BN * 128 + pg * 64 * 128, map, fb, p * C::PW, 0, T.hk,
+                                                    phys);
                                     }
+                                } else {
+                                    tma_load_4d(dst + p * BN * 128, map, fb, p * C::PW, j * a.block, T.hk, T.b);
                                 }
-                                ++ring;
                             }
+                            ++ring;
+                            return true;
+                        };
+                        // The MMA warps' order: S(0), then S(k+1) ahead of PV(k); the loads follow
+                        // it (K(0), then K(k+1) before V(k)), so the ring is consumed in the order
+                        // it is filled.
+                        const int kend = min(T.n_list, kb + kListChunkG);
+                        if (kb == 0) ok = issue(bars->lst[0], 0);
+                        for (int k = kb; ok && k < kend; ++k) {
+                            if (k + 1 < T.n_list)
+                                ok = issue(k + 1 < kend ? bars->lst[k + 1 - kb] : list_entry(a, T, k + 1), 0);
+                            if (ok) ok = issue(bars->lst[k - kb], 1);
                         }
                     }
                     ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
                 }
-                it.next(a);
             }
             if (lane == 0) {
                 if (bad) atomicOr(a.err, bad);
@@ -276,12 +271,10 @@ __global__ void __launch_bounds__(kThreadsG, 1)
                 const uint32_t aQ = smem_u32(smem + slot * C::Q_BYTES);
                 const uint32_t tS = tmem + slot * BN;
                 const uint32_t tO = tmem + 256 + slot * D;
-                uint32_t rbase = 0, qc = 0, pc = 0, sf = 0;
+                uint32_t rbase = 0, qc = 0, pc = 0, sf = 0, tn = 0;
                 bool ok = true, first_s = true;
-                UnitIter it;
-                it.init(blockIdx.x, gridDim.x, total_units);
-                it.next(a);
-                // S = Q K^T from ring index r (K of a block sits at 2k, its V at 2k + 1).
+                Tile T;
+                // S = Q K^T with K from ring position r.
                 auto mma_s = [&](uint32_t r) -> bool {
                     // S is overwritten: the softmax must have read the previous S.
                     if (!first_s) {
@@ -325,22 +318,28 @@ __global__ void __launch_bounds__(kThreadsG, 1)
                     tc_commit(&B.o_done[pb]);
                     return true;
                 };
-                while (ok && it.active) {
-                    const int n = it.T.n_list;
+                while (ok) {
+                    const int nt = tile_ring_get(bars->units, tn++, a, T, abort_flag);
+                    if (nt <= 0) {
+                        ok = nt == 0;
+                        break;
+                    }
+                    const int n = T.n_list;
                     ok = mbar_wait(&bars->q_full, qc & 1, abort_flag, a.err);
                     ++qc;
+                    // Ring positions of the unit (the producer's order K0, K1, V0, K2, V1, ...,
+                    // V(n-1)): K(k) at 2k - 1 for k >= 1, V(k) at 2k + 2 for k < n - 1, V(n - 1) at 2n - 1.
                     ok = ok && mma_s(rbase);
                     if (ok && n == 1) tc_commit(&bars->q_empty);
                     for (int k = 0; ok && k < n; ++k) {
                         // S(k+1) goes ahead of PV(k): it only needs the softmax to have read S(k).
                         if (k + 1 < n) {
-                            ok = mma_s(rbase + 2 * (k + 1));
+                            ok = mma_s(rbase + 2 * k + 1);
                             if (ok && k + 2 == n) tc_commit(&bars->q_empty);  // last S of the unit
                         }
-                        ok = ok && mma_pv(rbase + 2 * k + 1, k > 0);
+                        ok = ok && mma_pv(rbase + (k + 1 < n ? 2 * k + 2 : 2 * n - 1), k > 0);
                     }
                     rbase += 2 * n;
-                    it.next(a);
                 }
                 tc_commit(&B.drain);
                 volatile int no_abort = 0;
@@ -385,11 +384,10 @@ __global__ void __launch_bounds__(kThreadsG, 1)
     // Slot 0 takes the first turn: slot 1 hands it over once at the start.
     if (slot == 1) mbar_arrive(&bars->turn[0]);
     uint32_t turns = 0;
-    UnitIter it;
-    it.init(blockIdx.x, gridDim.x, total_units);
-    it.next(a);
-    while (ok && it.active) {
-        const Tile T = it.T;
+    uint32_t tn = 0;
+    while (ok) {
+        Tile T;
+        if (tile_ring_get_warp(bars->units, tn++, a, T, abort_flag, lane) <= 0) break;
         const int h = T.h + slot;
         float m_used = -INFINITY, l_run = 0.f;
         // The unit's list, 32 entries per warp-wide load (lane e: entry 32c + e), a chunk ahead of
@@ -568,7 +566,6 @@ __global__ void __launch_bounds__(kThreadsG, 1)
             a.lse[(static_cast<int64_t>(T.b) * a.Hq + h) * a.lse_stride + t_row] =
                 (m_used + __log2f(l_run) - kPScaleG) * 0.69314718055994531f;
         tc_fence_before();
-        it.next(a);
     }
     tc_fence_before();
     mbar_arrive(&bars->tmem_free);
@@ -578,6 +575,7 @@ template <bool PAGED>
 cudaError_t launch_group_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const AttnArgs& a,
                            cudaStream_t s) {
     using C = CfgG<true, 128, 128>;
+    if (a.tile_counter == nullptr) return cudaErrorInvalidValue;
     auto kern = attn_group_kernel<PAGED>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;

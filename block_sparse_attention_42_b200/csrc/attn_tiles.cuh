@@ -126,18 +126,26 @@ __device__ __forceinline__ void tile_ring_init(TileRing& r, int consumers) {
     }
 }
 
-// Producer, one thread: publishes the next non-empty tile at or after the counter (or -1) in
-// slot n % kTileRing.  False when the wait for the slot failed (nothing published).
-__device__ __forceinline__ bool tile_ring_put(TileRing& r, uint32_t n, const AttnArgs& a, int total_tiles, int& t,
-                                              volatile int* abort_flag) {
+// Producer, one thread: publishes, in slot n % kTileRing, the tile of the next counter value
+// c < total whose tile to_tile(c) is not empty (or -1 when none is left); t receives it.  The
+// counter runs over work units, to_tile maps a unit to the tile index the consumers decode
+// (the identity for per-head tiles).  False when the wait for the slot failed (nothing
+// published).
+struct TileIdentity {
+    __device__ __forceinline__ int operator()(int c) const { return c; }
+};
+template <class ToTile = TileIdentity>
+__device__ __forceinline__ bool tile_ring_put(TileRing& r, uint32_t n, const AttnArgs& a, int total, int& t,
+                                              volatile int* abort_flag, ToTile to_tile = ToTile()) {
     const uint32_t slot = n % kTileRing;
     if (!mbar_wait(&r.empty[slot], ((n / kTileRing) & 1) ^ 1, abort_flag, a.err)) return false;
     while (true) {
-        t = atomicAdd(a.tile_counter, 1);
-        if (t >= total_tiles) {
+        const int c = atomicAdd(a.tile_counter, 1);
+        if (c >= total) {
             t = -1;
             break;
         }
+        t = to_tile(c);
         const Tile U = decode_tile(a, t);
         if (U.valid && U.n_list > 0) break;
     }
