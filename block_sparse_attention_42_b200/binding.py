@@ -26,7 +26,7 @@ EXPORTS = ["bsa_tpd_budget", "bsa_score_workspace_bytes", "stem_score", "stem_se
            "bsa_prefill_paged", "bsa_last_error", "bsa_check_device_error", "stem_score_noalloc",
            "bsa_selftest_wait_timeout", "bsa_mask_workspace_bytes", "bsa_mask_to_lists", "bsa_prefill_mask",
            "bsa_validate_lists", "bsa_score_group_workspace_bytes", "stem_score_group", "bsa_prefill_group",
-           "bsa_prefill_skip", "bsa_score_select_workspace_bytes", "stem_score_select"]
+           "bsa_prefill_skip", "bsa_score_select_workspace_bytes", "stem_score_select", "bsa_prefill_paged_group"]
 
 
 class BsaError(RuntimeError):
@@ -69,6 +69,7 @@ def lib():
     L.bsa_prefill_skip.argtypes = [T, T, T, T, i32, i32, i32, i32, i32, i32, P, i32, P, i64, f32, f64, P, P, P]
     L.bsa_prefill_paged.argtypes = [T, T, P, P, i32, T, T, i32, i32, P, i32, i32, i32, i32, i32, P, i32, P, i64,
                                     f32, P, P]
+    L.bsa_prefill_paged_group.argtypes = L.bsa_prefill_paged.argtypes
     L.bsa_mask_workspace_bytes.argtypes = [i32, i32, i32]
     L.bsa_mask_workspace_bytes.restype = ctypes.c_size_t
     L.bsa_mask_to_lists.argtypes = [P, i64, i32, i32, i32, P, P, i64, P]
@@ -77,7 +78,7 @@ def lib():
     L.bsa_last_error.restype = ctypes.c_char_p
     L.bsa_check_device_error.argtypes = [P]
     L.bsa_selftest_wait_timeout.argtypes = [ctypes.c_uint64, P]
-    for name in ["stem_score", "stem_score_select", "stem_score_group", "bsa_prefill_group", "bsa_prefill_skip", "stem_score_noalloc", "stem_select", "bsa_prefill", "bsa_prefill_paged", "bsa_check_device_error",
+    for name in ["stem_score", "stem_score_select", "stem_score_group", "bsa_prefill_group", "bsa_prefill_skip", "stem_score_noalloc", "stem_select", "bsa_prefill", "bsa_prefill_paged", "bsa_prefill_paged_group", "bsa_check_device_error",
                  "bsa_selftest_wait_timeout", "bsa_mask_to_lists", "bsa_prefill_mask", "bsa_validate_lists"]:
         getattr(L, name).restype = ctypes.c_int
     _lib = L
@@ -375,7 +376,7 @@ def bsa_validate_lists(row_ptr, col_idx, nb_per_seq, allow_empty: bool = False):
 
 def bsa_prefill_paged(q, cu_seqlens, seqlens, k_cache, v_cache, page_table, block: int, row_ptr, col_idx,
                       softmax_scale: float = 0.0, out=None, lse=None, return_lse: bool = False, q_scale=1.0,
-                      k_scale=1.0, v_scale=1.0):
+                      k_scale=1.0, v_scale=1.0, _group: bool = False):
     """Paged-KV variant: q packed [sum N, Hq, d]; k_cache/v_cache [num_pages, page_size, Hkv, d]."""
     T, Hq, d = q.shape
     num_pages, page_size, Hkv, _ = k_cache.shape
@@ -387,12 +388,23 @@ def bsa_prefill_paged(q, cu_seqlens, seqlens, k_cache, v_cache, page_table, bloc
     if return_lse and lse is None:
         lse = torch.empty(B, Hq, max(seqlens), dtype=torch.float32, device=q.device)
     kc, vc = tensor_arg(k_cache, k_scale), tensor_arg(v_cache, v_scale)
-    st = lib().bsa_prefill_paged(tensor_arg(q, q_scale), tensor_arg(out), _ptr(cu_seqlens),
-                                 ctypes.c_void_p(sl.data_ptr()), B, kc, vc, num_pages, page_size, _ptr(page_table),
-                                 page_table.shape[-1], Hq, Hkv, d, block, _ptr(row_ptr), row_ptr.shape[-1],
-                                 _ptr(col_idx), col_idx.shape[-1], float(softmax_scale), _ptr(lse), _stream(q))
+    fn = lib().bsa_prefill_paged_group if _group else lib().bsa_prefill_paged
+    st = fn(tensor_arg(q, q_scale), tensor_arg(out), _ptr(cu_seqlens), ctypes.c_void_p(sl.data_ptr()), B, kc, vc,
+            num_pages, page_size, _ptr(page_table), page_table.shape[-1], Hq, Hkv, d, block, _ptr(row_ptr),
+            row_ptr.shape[-1], _ptr(col_idx), col_idx.shape[-1], float(softmax_scale), _ptr(lse), _stream(q))
     _check(st)
     return (out, lse) if return_lse else out
+
+
+def bsa_prefill_paged_group(q, cu_seqlens, seqlens, k_cache, v_cache, page_table, block: int, row_ptr, col_idx,
+                            softmax_scale: float = 0.0, out=None, lse=None, return_lse: bool = False, q_scale=1.0,
+                            k_scale=1.0, v_scale=1.0):
+    """bsa_prefill_paged with one list per KV-head group: col_idx [B, Hkv, max_k] (from stem_select
+    on stem_score_group's scores), shared by the group's query heads."""
+    if col_idx.shape[1] != k_cache.shape[2]:
+        raise ValueError("col_idx must be [B, Hkv, max_k]: one list per KV-head group")
+    return bsa_prefill_paged(q, cu_seqlens, seqlens, k_cache, v_cache, page_table, block, row_ptr, col_idx,
+                             softmax_scale, out, lse, return_lse, q_scale, k_scale, v_scale, _group=True)
 
 
 def bsa_check_device_error(device=None):

@@ -787,13 +787,16 @@ bsa_status_t bsa_prefill_mask(bsa_tensor_t q, bsa_tensor_t k, bsa_tensor_t v, bs
                           softmax_scale, lse, stream);
 }
 
-bsa_status_t bsa_prefill_paged(bsa_tensor_t q, bsa_tensor_t out, const int32_t* cu_seqlens, const int32_t* seqlens_host,
-                               int32_t B, bsa_tensor_t k_cache, bsa_tensor_t v_cache, int32_t num_pages,
-                               int32_t page_size, const int32_t* page_table, int32_t max_pages, int32_t Hq,
-                               int32_t Hkv, int32_t d, int32_t block, const int32_t* row_ptr,
-                               int32_t row_ptr_stride, const int32_t* col_idx, int64_t max_k, float softmax_scale,
-                               float* lse, cudaStream_t stream) {
-    NvtxRange nvtx_range("bsa_prefill_paged");
+namespace {
+
+// bsa_prefill_paged and bsa_prefill_paged_group: checks, tensor maps and the launch; `group`
+// selects one list per KV-head group (col_idx [B, Hkv, max_k]).
+bsa_status_t paged_launch(bsa_tensor_t q, bsa_tensor_t out, const int32_t* cu_seqlens, const int32_t* seqlens_host,
+                          int32_t B, bsa_tensor_t k_cache, bsa_tensor_t v_cache, int32_t num_pages,
+                          int32_t page_size, const int32_t* page_table, int32_t max_pages, int32_t Hq, int32_t Hkv,
+                          int32_t d, int32_t block, const int32_t* row_ptr, int32_t row_ptr_stride,
+                          const int32_t* col_idx, int64_t max_k, float softmax_scale, float* lse,
+                          cudaStream_t stream, bool group) {
     bsa_status_t st;
     if ((st = check_tensor(q, "q", false)) || (st = check_tensor(out, "out", false)) ||
         (st = check_tensor(k_cache, "k_cache", true)) || (st = check_tensor(v_cache, "v_cache", true)))
@@ -858,10 +861,43 @@ bsa_status_t bsa_prefill_paged(bsa_tensor_t q, bsa_tensor_t out, const int32_t* 
     a.lse = lse;
     a.lse_stride = n_max;
     a.err = err;
+    a.list_per_group = group ? 1 : 0;
     if (!(a.tile_counter = tile_counter(stream, &est))) return est;
-    cudaError_t e = launch_attn(fp8, true, tq, tk, tv, a, stream);
-    if (e != cudaSuccess) return cuda_fail(e, "bsa_prefill_paged launch");
+    // Group-shared lists: the GQA-packed kernel where it applies (BSA_ATTN_VARIANT still picks a
+    // per-head kernel for cross-checks), else the per-head kernels on the shared lists.
+    const char* var = std::getenv("BSA_ATTN_VARIANT");
+    const bool packed = group && attention_group_packed(fp8, a) && (!var || std::strcmp(var, "group") == 0);
+    cudaError_t e = packed ? launch_attention_group(fp8, true, tq, tk, tv, a, stream)
+                           : launch_attn(fp8, true, tq, tk, tv, a, stream);
+    if (e != cudaSuccess) return cuda_fail(e, group ? "bsa_prefill_paged_group launch" : "bsa_prefill_paged launch");
     return BSA_OK;
+}
+
+}  // namespace
+
+bsa_status_t bsa_prefill_paged(bsa_tensor_t q, bsa_tensor_t out, const int32_t* cu_seqlens, const int32_t* seqlens_host,
+                               int32_t B, bsa_tensor_t k_cache, bsa_tensor_t v_cache, int32_t num_pages,
+                               int32_t page_size, const int32_t* page_table, int32_t max_pages, int32_t Hq,
+                               int32_t Hkv, int32_t d, int32_t block, const int32_t* row_ptr,
+                               int32_t row_ptr_stride, const int32_t* col_idx, int64_t max_k, float softmax_scale,
+                               float* lse, cudaStream_t stream) {
+    NvtxRange nvtx_range("bsa_prefill_paged");
+    return paged_launch(q, out, cu_seqlens, seqlens_host, B, k_cache, v_cache, num_pages, page_size, page_table,
+                        max_pages, Hq, Hkv, d, block, row_ptr, row_ptr_stride, col_idx, max_k, softmax_scale, lse,
+                        stream, false);
+}
+
+bsa_status_t bsa_prefill_paged_group(bsa_tensor_t q, bsa_tensor_t out, const int32_t* cu_seqlens,
+                                     const int32_t* seqlens_host, int32_t B, bsa_tensor_t k_cache,
+                                     bsa_tensor_t v_cache, int32_t num_pages, int32_t page_size,
+                                     const int32_t* page_table, int32_t max_pages, int32_t Hq, int32_t Hkv,
+                                     int32_t d, int32_t block, const int32_t* row_ptr, int32_t row_ptr_stride,
+                                     const int32_t* col_idx, int64_t max_k, float softmax_scale, float* lse,
+                                     cudaStream_t stream) {
+    NvtxRange nvtx_range("bsa_prefill_paged_group");
+    return paged_launch(q, out, cu_seqlens, seqlens_host, B, k_cache, v_cache, num_pages, page_size, page_table,
+                        max_pages, Hq, Hkv, d, block, row_ptr, row_ptr_stride, col_idx, max_k, softmax_scale, lse,
+                        stream, true);
 }
 
 const char* bsa_last_error(void) { return g_last_error.c_str(); }

@@ -23,6 +23,8 @@
 //   warps 4-7   softmax of slot 0, warps 8-11 softmax of slot 1: one query row per thread (TMEM
 //               lane quadrant = warp % 4), as in the per-head kernels.
 // Per slot two P buffers: P(k) only waits for PV(k-2).
+// Paged K/V (bsa_prefill_paged_group): the producer loads a kept block as its 64-token pages
+// through the page table, as the per-head kernels do; Q and O are the packed varlen rows.
 // The two slots read the same blocks, so their S products land together and, left alone, their
 // exponential phases would run at the same time: the MUFU (16 ex2 per clock per SM) would be
 // shared while both exponentiate and idle while both do the rest of a block.  A token makes the
@@ -597,8 +599,8 @@ bool attention_group_packed(bool fp8, const AttnArgs& a) {
 
 cudaError_t launch_attention_group(bool fp8, bool paged, const CUtensorMap& tq, const CUtensorMap& tk,
                                    const CUtensorMap& tv, const AttnArgs& a, cudaStream_t s) {
-    if (!attention_group_packed(fp8, a) || paged) return cudaErrorInvalidValue;
-    return launch_group_t<false>(tq, tk, tv, a, s);
+    if (!attention_group_packed(fp8, a)) return cudaErrorInvalidValue;
+    return paged ? launch_group_t<true>(tq, tk, tv, a, s) : launch_group_t<false>(tq, tk, tv, a, s);
 }
 
 }  // namespace bsa

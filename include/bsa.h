@@ -22,7 +22,7 @@
  *   stem_score_select
  *                stem_score + stem_select in one call without the score matrix [same page,
  *                §二.2.1: no large intermediates].
- *   stem_score_group / bsa_prefill_group
+ *   stem_score_group / bsa_prefill_group / bsa_prefill_paged_group
  *                one list per KV-head group shared by its query heads, and attention that loads
  *                each kept K/V block once for two heads (an extension; the pages say nothing
  *                about grouped-query attention).
@@ -267,6 +267,22 @@ bsa_status_t bsa_prefill_paged(bsa_tensor_t q, bsa_tensor_t out, const int32_t* 
                                int32_t Hkv, int32_t d, int32_t block, const int32_t* row_ptr,
                                int32_t row_ptr_stride, const int32_t* col_idx, int64_t max_k,
                                float softmax_scale, float* lse, cudaStream_t stream);
+
+/* bsa_prefill_paged with group-shared lists: col_idx is [B, Hkv, max_k], one list per KV-head
+ * group shared by the group's query heads (row_ptr [B, row_ptr_stride] as stem_select writes
+ * it for stem_score_group's scores).  FP8 at d = 128, block 128, with G even, runs the
+ * GQA-packed kernel of bsa_prefill_group on the page pool: one CTA serves two query heads of
+ * a group for a query block and loads each kept block's pages once for both.  Every other
+ * shape runs the per-head paged kernel on the shared lists.  Arguments, page rules, outputs
+ * and errors otherwise as in bsa_prefill_paged.  (An extension: the pages select per query
+ * head and say nothing about grouped-query attention.) */
+bsa_status_t bsa_prefill_paged_group(bsa_tensor_t q, bsa_tensor_t out, const int32_t* cu_seqlens,
+                                     const int32_t* seqlens_host, int32_t B, bsa_tensor_t k_cache,
+                                     bsa_tensor_t v_cache, int32_t num_pages, int32_t page_size,
+                                     const int32_t* page_table, int32_t max_pages, int32_t Hq,
+                                     int32_t Hkv, int32_t d, int32_t block, const int32_t* row_ptr,
+                                     int32_t row_ptr_stride, const int32_t* col_idx, int64_t max_k,
+                                     float softmax_scale, float* lse, cudaStream_t stream);
 
 /* stem_score without a workspace argument, for callers that cannot allocate device memory:
  * for example a plain C host program that links only this library and has no device

@@ -106,6 +106,10 @@ def test_argument_errors_return_status(lib):
     sl = (ctypes.c_int32 * 1)(1024)
     assert lib.bsa_prefill_paged(_t(), _t(), P(1), sl, 1, _t(), _t(), 100, 32, P(1), 16, 8, 8, 128, 128, P(1), 9,
                                  P(1), 36, 0.0, None, None) == 2
+    assert lib.bsa_prefill_paged_group(_t(), _t(), P(1), sl, 1, _t(), _t(), 100, 32, P(1), 16, 8, 8, 128, 128, P(1),
+                                       9, P(1), 36, 0.0, None, None) == 2
+    assert lib.bsa_prefill_paged_group(_t(), _t(), None, sl, 1, _t(), _t(), 100, 64, P(1), 16, 8, 8, 128, 128, P(1),
+                                       9, P(1), 36, 0.0, None, None) == 1
     # block-mask input: stride a multiple of 16 and >= nb, a 16-byte aligned mask, room for the
     # lists; nb at most 2048
     ws_need = lib.bsa_mask_workspace_bytes(1, 8, 8)
