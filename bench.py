@@ -558,6 +558,31 @@ def run_ours(args, rank, world, device):
                         "select_ms": sel_ms, "bsa_prefill_group_ms": attn_g_ms, "effective_flop": g_flop,
                         "effective_tflops": g_flop / (attn_g_ms * 1e-3) / 1e12,
                         "per_head_bsa_prefill_ms": res["attn_ms"], "reps": reps}
+        # The same K/V in a pool of 64-token pages placed by a seeded permutation (the serving
+        # engine's cache layout), through bsa_prefill_paged_group: same lists, same kernel.
+        if B == 1 and N % 64 == 0:
+            npg = N // 64
+            perm = torch.randperm(npg, generator=torch.Generator().manual_seed(7)).to(device)
+            k_pool = torch.empty(npg, 64, Hkv, D, dtype=k.dtype, device=device)
+            v_pool = torch.empty_like(k_pool)
+            k_pool[perm] = k[0].reshape(npg, 64, Hkv, D)
+            v_pool[perm] = v[0].reshape(npg, 64, Hkv, D)
+            page_table = perm.to(torch.int32).view(1, npg)
+            cu = torch.tensor([0, N], dtype=torch.int32, device=device)
+            g_outp = torch.empty(N, Hq, D, dtype=torch.bfloat16, device=device)
+
+            def g_attn_paged():
+                bsa.bsa_prefill_paged_group(q[0], cu, [N], k_pool, v_pool, page_table, w.block, g_rp, g_ci,
+                                            out=g_outp, **scale_kw)
+
+            paged_ms = _time_calls(g_attn_paged, reps, stream)
+            bsa.bsa_check_device_error(device)
+            res["group"].update({"paged_group_ms": paged_ms,
+                                 "paged_group_tflops": g_flop / (paged_ms * 1e-3) / 1e12,
+                                 "paged_equals_contiguous": bool(torch.equal(g_outp.view(torch.int16),
+                                                                             g_out[0].view(torch.int16))),
+                                 "paged_layout": f"{npg} pages of 64 tokens, seeded permutation"})
+            del k_pool, v_pool, g_outp
         del g_scores, g_ws, g_rp, g_ci, g_out
 
     # Score + select in one call without the score matrix: same lists, timed like select_ms.
