@@ -818,7 +818,11 @@ def main():
                          "peak_source": f"{src} bf16 {'sustained' if 'bf16_tflops_sustained' in pk else 'burst'}"
                                         f"{' x2 (fp8/bf16 nominal ratio)' if fp8 else ''}",
                          "traffic": attn_traffic(fp8, res["B"], res["N"], res["Hq"], res["Hkv"], res["D"]),
-                         "traffic_source": "ncu dram bytes of the fp8-32k capture, scaled by tokens"},
+                         "traffic_source": "ncu dram bytes of the fp8-32k capture, scaled by tokens",
+                         # the same against the burst GEMM figure (measured near the maximum clock,
+                         # where this kernel runs; the sustained figure was measured power-capped)
+                         "peak_burst": pk["bf16_tflops"] * (2.0 if fp8 else 1.0),
+                         "frac_of_burst_peak": attn_ach / (pk["bf16_tflops"] * (2.0 if fp8 else 1.0))},
             # The bound that binds for E4M3 attention: the exponentials.  Every kept 128-key
             # block needs block x block exp2 per query row tile; the MUFU unit does 16 per clock
             # per SM (measured with a throughput probe on this machine), so the peak is
