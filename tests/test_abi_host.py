@@ -173,3 +173,22 @@ def test_block_mask_buffer_and_argument_checks():
         binding._mask_arg(torch.zeros(1, 2, 20, 32, dtype=torch.uint8)[..., ::2], 1, 2, 20)  # strided columns
     with pytest.raises(ValueError):
         binding._mask_arg(torch.zeros(1, 20, 2, 32, dtype=torch.uint8).transpose(1, 2), 1, 2, 20)  # heads not outer
+
+
+def test_group_wrappers_refuse_per_head_lists():
+    """bsa_prefill_group and bsa_prefill_paged_group take one list per KV-head group
+    (col_idx [B, Hkv, max_k]); per-head lists are refused before anything is launched (CPU
+    tensors)."""
+    from block_sparse_attention_42_b200 import binding
+    B, N, Hq, Hkv, d = 1, 256, 8, 2, 128
+    q = torch.zeros(B, N, Hq, d, dtype=torch.bfloat16)
+    k = torch.zeros(B, N, Hkv, d, dtype=torch.bfloat16)
+    rp = torch.zeros(B, 3, dtype=torch.int32)
+    per_head = torch.zeros(B, Hq, 3, dtype=torch.int32)
+    with pytest.raises(ValueError):
+        binding.bsa_prefill_group(q, k, k, 128, rp, per_head)
+    kc = torch.zeros(4, 64, Hkv, d, dtype=torch.bfloat16)
+    pt = torch.arange(4, dtype=torch.int32).view(1, 4)
+    cu = torch.tensor([0, N], dtype=torch.int32)
+    with pytest.raises(ValueError):
+        binding.bsa_prefill_paged_group(q[0], cu, [N], kc, kc, pt, 128, rp, per_head)
